@@ -1,0 +1,134 @@
+// epilogue.cuh - fused GEMM epilogues of the DiT block.
+//
+// Every Linear of the block ends in one of these, applied by the thread that owns
+// one output row to 32 consecutive columns at a time (columns come in groups of
+// 128 = one attention head):
+//   EPI_STORE  y = acc + bias                              (patch embed, head, v-part)
+//   EPI_GELU   y = gelu_tanh(acc + bias)                    (FFN1)
+//   EPI_RESID  x[row] += gate[stream] * (acc + bias)        (O-proj, cross-O, FFN2; gate
+//                                                            null means 1: ungated, R8)
+//   EPI_NORM   y = acc + bias; on "normed" columns the partial sum of y^2 over the
+//              head's 128 columns goes to ssq[row, group] and y *= gain (cross-attn
+//              q and k: full-width RMSNorm split per head, reading R4)
+//   EPI_QKV    as EPI_NORM for the q and k sections, plus 3D rotary on adjacent
+//              pairs (2d, 2d+1) of q and k, and a head-major scatter of q, k, v to
+//              [3][B][heads][L][128] (reading R3).
+// The RMS factor r = (sum(ssq)/D + eps)^-1/2 itself is applied later, inside the
+// attention kernels, to the scores: r is one scalar per row and both the gain and
+// the rotation are linear per channel, so RoPE(g * r * y) = r * RoPE(g * y).
+#pragma once
+
+#include "common.cuh"
+
+namespace fh {
+
+enum EpiKind { EPI_STORE = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_NORM = 3, EPI_QKV = 4 };
+
+struct EpiParams {
+  const float* bias;      // [N]
+  void* out;              // output base (row-major [M, ldo] unless EPI_QKV)
+  long ldo;
+  float* resid;           // EPI_RESID: float32 residual [M, ldr]
+  long ldr;
+  const float* gate;      // EPI_RESID: gate[(row / rows_per_batch) * gate_bstride + col], or null
+  long gate_bstride;
+  int rows_per_batch;     // tokens per stream (L)
+  const float* gain;      // EPI_NORM/QKV: gain[col] on normed columns
+  float* ssq;             // EPI_NORM/QKV: ssq[row * ssq_ld + col / 128] on normed columns
+  int ssq_ld;
+  int norm_period;        // column c is normed iff (c % norm_period) < norm_count
+  int norm_count;
+  const float2* rope;     // EPI_QKV: (cos, sin) [rows_per_batch, 64]
+  int dim;                // EPI_QKV: width D of each of the q, k, v sections
+  long sec_stride;        // EPI_QKV: elements per section = B * heads * L * 128
+};
+
+__device__ __forceinline__ bool epi_normed(const EpiParams& p, int col) {
+  return (col % p.norm_period) < p.norm_count;
+}
+
+template <int KIND, typename OutT>
+__device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0, float (&v)[32],
+                                          float& ssq_acc) {
+  const float* b = p.bias + col0;
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    float4 bb = *reinterpret_cast<const float4*>(b + j);
+    v[j] += bb.x; v[j + 1] += bb.y; v[j + 2] += bb.z; v[j + 3] += bb.w;
+  }
+  if constexpr (KIND == EPI_STORE || KIND == EPI_GELU) {
+    if constexpr (KIND == EPI_GELU) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+    }
+    OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)row * p.ldo + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) store8(dst + j, v + j);
+  } else if constexpr (KIND == EPI_RESID) {
+    float* r = p.resid + (long)row * p.ldr + col0;
+    if (p.gate) {
+      const float* g = p.gate + (long)(row / p.rows_per_batch) * p.gate_bstride + col0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 gg = *reinterpret_cast<const float4*>(g + j);
+        v[j] *= gg.x; v[j + 1] *= gg.y; v[j + 2] *= gg.z; v[j + 3] *= gg.w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      float4 x = *reinterpret_cast<float4*>(r + j);
+      x.x += v[j]; x.y += v[j + 1]; x.z += v[j + 2]; x.w += v[j + 3];
+      *reinterpret_cast<float4*>(r + j) = x;
+    }
+  } else {  // EPI_NORM, EPI_QKV
+    const bool normed = epi_normed(p, col0);
+    if (normed) {
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) s = fmaf(v[j], v[j], s);
+      ssq_acc += s;
+      const float* g = p.gain + col0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 gg = *reinterpret_cast<const float4*>(g + j);
+        v[j] *= gg.x; v[j + 1] *= gg.y; v[j + 2] *= gg.z; v[j + 3] *= gg.w;
+      }
+    }
+    if constexpr (KIND == EPI_NORM) {
+      OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)row * p.ldo + col0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) store8(dst + j, v + j);
+    } else {
+      const int l = row % p.rows_per_batch;
+      const int bidx = row / p.rows_per_batch;
+      const int sec = col0 / p.dim;
+      const int cin = col0 - sec * p.dim;
+      const int head = cin >> 7;
+      const int d0 = cin & 127;
+      if (normed) {
+        const float2* rt = p.rope + (long)l * 64 + (d0 >> 1);
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float2 cs = rt[j >> 1];
+          float x0 = v[j], x1 = v[j + 1];
+          v[j] = x0 * cs.x - x1 * cs.y;
+          v[j + 1] = x0 * cs.y + x1 * cs.x;
+        }
+      }
+      const int heads = p.dim >> 7;
+      OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)sec * p.sec_stride +
+                  (((long)bidx * heads + head) * p.rows_per_batch + l) * 128 + d0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) store8(dst + j, v + j);
+    }
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ void epi_group_end(const EpiParams& p, int row, int gcol0, float ssq_acc) {
+  if constexpr (KIND == EPI_NORM || KIND == EPI_QKV) {
+    if (epi_normed(p, gcol0)) p.ssq[(long)row * p.ssq_ld + (gcol0 >> 7)] = ssq_acc;
+  }
+}
+
+}  // namespace fh

@@ -1,0 +1,258 @@
+// gemm_tc.cu - bf16 tensor-core GEMM with fused epilogues for sm_100a.
+//
+// out[M, N] = epilogue(A[M, K] * W[N, K]^T): A is an activation (bf16, row-major,
+// K contiguous), W a Linear weight in nn.Linear layout [out, in] (bf16, K
+// contiguous). This is every dense contraction of the DiT: patch embed, QKV,
+// O-proj, cross-Q, cross-KV, cross-O, FFN1, FFN2 and the head.
+//
+// Design (one CTA per SM, persistent over 128 x BN output tiles):
+//   warp 0     TMA producer: one thread streams 128x64 A and BNx64 W tiles with
+//              the 128-byte swizzle into a STAGES-deep shared-memory ring
+//              (per-CTA loads; no cluster multicast).
+//   warp 1     allocates 2*BN TMEM columns and, from one thread, issues
+//              tcgen05.mma (M=128, N=BN, K=16, fp32 accumulate in TMEM); each
+//              stage is released by tcgen05.commit to its "empty" mbarrier and
+//              each finished tile by a commit to its accumulator's "full" barrier.
+//   warps 2-5  epilogue: tcgen05.ld of 32 columns at a time (warp w reads TMEM
+//              lanes 32*(w%4)..+31 = its 32 output rows), the fused epilogue,
+//              direct 16-byte stores. Two accumulators alternate, so the
+//              epilogue of tile i overlaps the MMAs of tile i+1.
+// Every wait is bounded (FH_WAIT_LIMIT_NS); on expiry the CTA latches an error
+// bit, lets the producer's in-flight copies land, frees TMEM and exits.
+#include <cstdio>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace fh {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+
+template <int BN>
+struct TcShape {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > FH_WAIT_LIMIT_NS) return false;
+  }
+  return true;
+}
+
+template <int BN, int KIND, typename OutT>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
+                   int N, int K, EpiParams ep, unsigned* err) {
+  using S = TcShape<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::STAGES * S::STAGE_BYTES);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* tfull = empty + S::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_m = (M + BM - 1) / BM;
+  const int num_n = N / BN;
+  const int ntiles = num_m * num_n;
+  const int nk = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 2 * BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      long issues = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int m0 = (tile % num_m) * BM;
+        const int n0 = (tile / num_m) * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) goto producer_done;
+          uint8_t* sa = smem + stage * S::STAGE_BYTES;
+          mbar_expect_tx(&full[stage], S::STAGE_BYTES);
+          tma_load_2d(&tmA, &full[stage], sa, kb * BK, m0);
+          tma_load_2d(&tmB, &full[stage], sa + S::A_BYTES, kb * BK, n0);
+          ++issues;
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      if (*abort_flag) {
+        // let every copy this thread started land before the CTA's shared memory goes away
+        for (int s = 0; s < S::STAGES; ++s) {
+          if (issues <= 0) break;
+          int st = stage - 1 - s;
+          uint32_t ph = phase;
+          if (st < 0) {
+            st += S::STAGES;
+            ph ^= 1u;
+          }
+          drain_wait(&full[st], ph);
+          --issues;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
+        const int acc = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + S::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_f16(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32), idesc,
+                       (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    int local = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+      if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld below is warp-collective
+      tc_fence_after();
+      const int m0 = (tile % num_m) * BM;
+      const int n0 = (tile / num_m) * BN;
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int g = 0; g < BN; g += 128) {
+        float ssq = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          float v[32];
+          tmem_ld32(tb + g + c, v);
+          tc_wait_ld();
+          if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
+        }
+        if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+template <int BN, int KIND, typename OutT>
+cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, const EpiParams& ep,
+                      unsigned* err, int num_sms, cudaStream_t st) {
+  using S = TcShape<BN>;
+  const int tiles = ((M + BM - 1) / BM) * (N / BN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  gemm_tc_kernel<BN, KIND, OutT><<<grid, 192, S::SMEM, st>>>(a, b, M, N, K, ep, err);
+  return cudaGetLastError();
+}
+
+template <int BN, int KIND, typename OutT>
+cudaError_t prepare_tc() {
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)TcShape<BN>::SMEM);
+}
+
+}  // namespace
+
+cudaError_t gemm_tc_prepare() {
+  const cudaError_t es[] = {
+      prepare_tc<128, EPI_STORE, bf16>(), prepare_tc<256, EPI_STORE, bf16>(), prepare_tc<128, EPI_GELU, bf16>(),
+      prepare_tc<256, EPI_GELU, bf16>(),  prepare_tc<128, EPI_NORM, bf16>(),  prepare_tc<256, EPI_NORM, bf16>(),
+      prepare_tc<128, EPI_QKV, bf16>(),   prepare_tc<256, EPI_QKV, bf16>(),   prepare_tc<128, EPI_RESID, bf16>(),
+      prepare_tc<256, EPI_RESID, bf16>(), prepare_tc<128, EPI_STORE, float>(), prepare_tc<256, EPI_STORE, float>()};
+  for (cudaError_t e : es)
+    if (e != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int bn, int kind,
+                    bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st) {
+#define FH_TC_CASE(BNV, KV, OT)                                          \
+  if (bn == BNV && kind == KV) return launch_tc<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st);
+  if (out_bf16) {
+    FH_TC_CASE(128, EPI_STORE, bf16)
+    FH_TC_CASE(256, EPI_STORE, bf16)
+    FH_TC_CASE(128, EPI_GELU, bf16)
+    FH_TC_CASE(256, EPI_GELU, bf16)
+    FH_TC_CASE(128, EPI_NORM, bf16)
+    FH_TC_CASE(256, EPI_NORM, bf16)
+    FH_TC_CASE(128, EPI_QKV, bf16)
+    FH_TC_CASE(256, EPI_QKV, bf16)
+    FH_TC_CASE(128, EPI_RESID, bf16)
+    FH_TC_CASE(256, EPI_RESID, bf16)
+  } else {
+    FH_TC_CASE(128, EPI_STORE, float)
+    FH_TC_CASE(256, EPI_STORE, float)
+  }
+#undef FH_TC_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fh

@@ -1,0 +1,82 @@
+// kernels.h - host-side launchers of the library's kernels (internal interface).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fh {
+
+typedef __nv_bfloat16 bf16;
+struct EpiParams;
+
+// bf16 tensor-core GEMM (gemm_tc.cu): out = epilogue(A[M,K] * W[N,K]^T); `a`, `b`
+// are TMA maps of A (box 64 x 128) and W (box 64 x bn) with the 128-byte swizzle.
+// N % bn == 0, K % 64 == 0.
+cudaError_t gemm_tc_prepare();  // sets the kernels' shared-memory attributes on the current device
+cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int bn, int kind,
+                    bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st);
+
+// fp32 CUDA-core GEMM (misc.cu) with the same epilogues; N % 128 == 0.
+cudaError_t gemm_simt(const float* A, long lda, const float* W, long ldw, int M, int N, int K, int kind,
+                      const EpiParams& ep, cudaStream_t st);
+
+// self-attention (attention.cu). q/k/v: [B, heads, L, 128]; out [B*L, heads*128];
+// ssq [B*L, ssq_ld] holds per-head partial sums of squares, q heads then k heads.
+cudaError_t attn_tc_prepare();
+cudaError_t attn_tc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const float* ssq,
+                    int ssq_ld, int batch, int heads, int L, float eps, bf16* out, unsigned* err,
+                    cudaStream_t st);
+template <typename T>
+cudaError_t attn_simt(const T* q, const T* k, const T* v, const float* ssq, int ssq_ld, int batch, int heads,
+                      int L, float eps, T* out, cudaStream_t st);
+
+// per-frame audio cross-attention (misc.cu).
+// q [B*L, D] row-major with ssq_q [B*L, heads]; keys/values: rows (b*F + f)*A + a of
+// kv (row stride ldkv), key columns at koff, value columns at voff, with key partial
+// sums of squares ssq_k[row * ssq_k_ld + ssq_k_off + h]. out [B*L, D].
+template <typename T>
+cudaError_t cross_attn(const T* q, const float* ssq_q, const T* kv, long ldkv, int koff, int voff,
+                       const float* ssq_k, int ssq_k_ld, int ssq_k_off, int batch, int heads, int L, int F, int A,
+                       float eps, T* out, cudaStream_t st);
+
+// row norms (misc.cu): out[row] = norm(x[row]) then
+//   mode 0: LayerNorm, * (1 + scale[b]) + shift[b]   (scale/shift rows of stride mod_bstride)
+//   mode 1: LayerNorm, * w + bb                       (learned affine)
+//   mode 2: RMSNorm,   * (1 + scale[b]) + shift[b]
+template <typename T>
+cudaError_t norm_rows(const float* x, T* out, int M, int D, int rows_per_batch, int mode, const float* shift,
+                      const float* scale, long mod_bstride, const float* w, const float* bb, float eps,
+                      cudaStream_t st);
+
+// timestep conditioning (misc.cu)
+struct TVals {
+  float t[8];
+};
+cudaError_t time_sinusoid(float* out, int batch, TVals tv, int dim, cudaStream_t st);
+template <typename WT>
+cudaError_t gemv(const WT* W, const float* x, const float* bias, float* y, int N, int K, int batch, int silu_in,
+                 int silu_out, cudaStream_t st);
+// mods[b][k][i][c] = table[k][i][c] + e0[b][i][c]; hmods[b][i][c] = htable[i][c] + e[b][c]
+cudaError_t assemble_mods(const float* table, const float* e0, const float* htable, const float* e, float* mods,
+                          float* hmods, int batch, int blocks, int D, cudaStream_t st);
+
+// latents (misc.cu). Channel-first [B, C, F*H*W] <-> token-major rows.
+template <typename T>
+cudaError_t prep_tokens(const float* x, const float* ref, const float* motion, int pin_frames, float* lat, T* tok,
+                        int batch, int C, int L, int HW, cudaStream_t st);
+template <typename T>
+cudaError_t euler_step(float* lat, const float* v, float dsig, int pinned_tokens, T* tok, int batch, int C, int L,
+                       cudaStream_t st);
+cudaError_t tokens_to_latent(const float* tok, float* out, int batch, int C, int L, cudaStream_t st);
+
+// seeded weights (misc.cu): element (r, c) of tensor `tid` -> dst[r * ld + c]
+// kind 0: z * 1/sqrt(fan) (computed as z / sqrt(fan)); 1: 1 + 0.1 z; 2: 0.1 z
+template <typename T>
+cudaError_t gen_tensor(T* dst, long rows, long cols, long ld, uint64_t seed, int tid, int kind, int fan,
+                       bool round_bf16, cudaStream_t st);
+cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st);
+cudaError_t fill_f32(float* p, long n, float v, cudaStream_t st);
+
+}  // namespace fh

@@ -1,0 +1,549 @@
+// misc.cu - CUDA-core kernels of the DiT hot path: row norms with adaLN
+// modulation, per-frame audio cross-attention, timestep conditioning, latent
+// layout/Euler/motion pinning, the seeded weight generator, and the fp32 GEMM of
+// the fp32 configuration.
+#include <math.h>
+
+#include "epilogue.cuh"
+#include "kernels.h"
+
+namespace fh {
+
+namespace {
+
+// ------------------------------------------------------------------ row norms
+// One warp per row; D = 128 * NV floats held in registers (float4 per lane per step).
+// Mode 0 / 2: the adaLN modulate h = n(x) * (1 + scale) + shift of the Wan-style
+// block (reading R1) and of the output norm (headMods, gizai:flashhead Types >
+// FlashHead, reading R9); mode 1: the learned-affine LayerNorm before the audio
+// cross-attention (reading R7). Biased variance, eps inside the root (R2).
+template <typename T, int NV>
+__global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ out, int M, int rows_per_batch,
+                                 int mode, const float* __restrict__ shift, const float* __restrict__ scale,
+                                 long mod_bstride, const float* __restrict__ w, const float* __restrict__ bb,
+                                 float eps) {
+  constexpr int D = NV * 128;
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (long)row * D);
+  float4 v[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) v[i] = xr[lane + 32 * i];
+  float mu = 0.f, rstd;
+  if (mode != 2) {
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    mu = warp_sum(s) * (1.f / D);
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float a = v[i].x - mu, b = v[i].y - mu, c = v[i].z - mu, d = v[i].w - mu;
+      q += (a * a + b * b) + (c * c + d * d);
+    }
+    rstd = rsqrtf(warp_sum(q) * (1.f / D) + eps);
+  } else {
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) q += (v[i].x * v[i].x + v[i].y * v[i].y) + (v[i].z * v[i].z + v[i].w * v[i].w);
+    rstd = rsqrtf(warp_sum(q) * (1.f / D) + eps);
+  }
+  const long mb = (long)(row / rows_per_batch) * mod_bstride;
+  T* orow = out + (long)row * D;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int col = (lane + 32 * i) * 4;
+    float y[4] = {(v[i].x - mu) * rstd, (v[i].y - mu) * rstd, (v[i].z - mu) * rstd, (v[i].w - mu) * rstd};
+    float4 a, c;
+    if (mode == 1) {
+      a = *reinterpret_cast<const float4*>(w + col);
+      c = *reinterpret_cast<const float4*>(bb + col);
+    } else {
+      a = *reinterpret_cast<const float4*>(scale + mb + col);
+      c = *reinterpret_cast<const float4*>(shift + mb + col);
+      a.x += 1.f; a.y += 1.f; a.z += 1.f; a.w += 1.f;
+    }
+    y[0] = y[0] * a.x + c.x;
+    y[1] = y[1] * a.y + c.y;
+    y[2] = y[2] * a.z + c.z;
+    y[3] = y[3] * a.w + c.w;
+    if constexpr (sizeof(T) == 2) {
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&h0);
+      u.y = *reinterpret_cast<uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(orow + col) = u;
+    } else {
+      *reinterpret_cast<float4*>(orow + col) = make_float4(y[0], y[1], y[2], y[3]);
+    }
+  }
+}
+
+// ------------------------------------------------------ per-frame cross-attention
+// A token of latent frame f attends to frame f's A audio tokens only (gizai:flashhead,
+// opening paragraph: 5 latent frames of 32 audio tokens; reading R5). One CTA per
+// (frame, head, stream) stages that frame's keys/values (fp32) and key RMS factors in
+// shared memory; one query per thread.
+template <typename T, int A>
+__global__ void __launch_bounds__(128) cross_attn_kernel(const T* __restrict__ q, const float* __restrict__ ssq_q,
+                                                         const T* __restrict__ kv, long ldkv, int koff, int voff,
+                                                         const float* __restrict__ ssq_k, int ssq_k_ld,
+                                                         int ssq_k_off, int heads, int L, int F, float eps,
+                                                         float scale, T* __restrict__ out) {
+  __shared__ float ks[A][129];
+  __shared__ float vs[A][128];
+  __shared__ float rks[A];
+  const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int D = heads * 128;
+  const float inv_d = 1.f / (float)D;
+  const long kv_row0 = ((long)b * F + f) * A;
+  for (int idx = threadIdx.x; idx < A * 128; idx += blockDim.x) {
+    const int a = idx >> 7, d = idx & 127;
+    const T* r = kv + (kv_row0 + a) * ldkv;
+    ks[a][d] = to_f(r[koff + h * 128 + d]);
+    vs[a][d] = to_f(r[voff + h * 128 + d]);
+  }
+  for (int a = threadIdx.x; a < A; a += blockDim.x) {
+    const float* p = ssq_k + (kv_row0 + a) * ssq_k_ld + ssq_k_off;
+    float s = 0.f;
+    for (int i = 0; i < heads; ++i) s += p[i];
+    rks[a] = rsqrtf(s * inv_d + eps);
+  }
+  __syncthreads();
+  const int HW = L / F;
+  for (int n = threadIdx.x; n < HW; n += blockDim.x) {
+    const long row = (long)b * L + (long)f * HW + n;
+    const float* pq = ssq_q + row * heads;
+    float sq = 0.f;
+    for (int i = 0; i < heads; ++i) sq += pq[i];
+    const float rq = rsqrtf(sq * inv_d + eps) * scale;
+    const T* qr = q + row * D + h * 128;
+    float s[A];
+#pragma unroll
+    for (int a = 0; a < A; ++a) s[a] = 0.f;
+#pragma unroll 1
+    for (int d0 = 0; d0 < 128; d0 += 8) {
+      float qv[8];
+      load8(qr + d0, qv);
+#pragma unroll
+      for (int a = 0; a < A; ++a) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s[a] = fmaf(qv[e], ks[a][d0 + e], s[a]);
+      }
+    }
+    float m = -INFINITY;
+#pragma unroll
+    for (int a = 0; a < A; ++a) {
+      s[a] *= rq * rks[a];
+      m = fmaxf(m, s[a]);
+    }
+    float z = 0.f;
+#pragma unroll
+    for (int a = 0; a < A; ++a) {
+      s[a] = expf(s[a] - m);
+      z += s[a];
+    }
+    const float iz = 1.f / z;
+    T* orow = out + row * D + h * 128;
+#pragma unroll 1
+    for (int d0 = 0; d0 < 128; d0 += 8) {
+      float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int a = 0; a < A; ++a) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = fmaf(s[a], vs[a][d0 + e], o[e]);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] *= iz;
+      store8(orow + d0, o);
+    }
+  }
+}
+
+// ------------------------------------------------------------ conditioning
+// 256-dim sinusoid of tau = 1000 t: [cos(tau w_k) | sin(tau w_k)], w_k = 10000^(-k/128)
+// (reading R10 of the timestep embedding that yields the per-step modulations,
+// gizai:flashhead Types > FlashHead, field headMods).
+__global__ void time_sinusoid_kernel(float* out, int batch, TVals tv, int dim) {
+  const int half = dim / 2;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= batch * dim) return;
+  const int b = idx / dim, k = idx % dim;
+  const int kk = k < half ? k : k - half;
+  const double w = pow(10000.0, -(double)kk / (double)half);
+  const double ang = 1000.0 * (double)tv.t[b] * w;
+  out[idx] = (float)(k < half ? cos(ang) : sin(ang));
+}
+
+// y[b, n] = act(sum_k W[n, k] * act_in(x[b, k]) + bias[n]); one warp per output.
+template <typename WT>
+__global__ void gemv_kernel(const WT* __restrict__ W, const float* __restrict__ x, const float* __restrict__ bias,
+                            float* __restrict__ y, int N, int K, int batch, int silu_in, int silu_out) {
+  extern __shared__ float xs[];
+  for (int i = threadIdx.x; i < batch * K; i += blockDim.x) {
+    const float v = x[i];
+    xs[i] = silu_in ? silu(v) : v;
+  }
+  __syncthreads();
+  const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (n >= N) return;
+  float acc[8];
+  for (int b = 0; b < batch; ++b) acc[b] = 0.f;
+  const WT* wr = W + (long)n * K;
+  for (int k = lane; k < K; k += 32) {
+    const float wv = to_f(wr[k]);
+    for (int b = 0; b < batch; ++b) acc[b] = fmaf(wv, xs[b * K + k], acc[b]);
+  }
+  for (int b = 0; b < batch; ++b) {
+    float s = warp_sum(acc[b]);
+    if (lane == 0) {
+      s += bias[n];
+      y[(long)b * N + n] = silu_out ? silu(s) : s;
+    }
+  }
+}
+
+__global__ void assemble_mods_kernel(const float* __restrict__ table, const float* __restrict__ e0,
+                                     const float* __restrict__ htable, const float* __restrict__ e,
+                                     float* __restrict__ mods, float* __restrict__ hmods, int batch, int blocks,
+                                     int D) {
+  const long per = (long)blocks * 6 * D;
+  const long total = (long)batch * per;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total + (long)batch * 2 * D;
+       i += (long)gridDim.x * blockDim.x) {
+    if (i < total) {
+      const long b = i / per, r = i % per;
+      const long ic = r % (6L * D);  // (i, c) within the block
+      mods[i] = table[r] + e0[b * 6L * D + ic];
+    } else {
+      const long j = i - total;
+      const long b = j / (2L * D), r = j % (2L * D);
+      hmods[j] = htable[r] + e[b * D + (r % D)];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ latents
+// Channel-first latents [B, C, L] -> token-major rows: lat[b*L+n][c] (float32, optional)
+// and the patch-embed input tok[b*L+n] = [x | ref] in T (the noisy latent's channels
+// first, reading R16). Frames below pin_frames take the motion latent (reading R14).
+template <typename T>
+__global__ void prep_tokens_kernel(const float* __restrict__ x, const float* __restrict__ ref,
+                                   const float* __restrict__ motion, int pin_frames, float* __restrict__ lat,
+                                   T* __restrict__ tok, int C, int L, int HW) {
+  __shared__ float tx[32][33];
+  __shared__ float tr[32][33];
+  const int b = blockIdx.z;
+  const int n0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+  const int pinned = pin_frames * HW;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, n = n0 + threadIdx.x;
+    float xv = 0.f, rv = 0.f;
+    if (n < L) {
+      const long src = ((long)b * C + c) * L + n;
+      xv = (motion != nullptr && n < pinned) ? motion[((long)b * C + c) * pinned + n] : x[src];
+      rv = ref[src];
+    }
+    tx[i][threadIdx.x] = xv;
+    tr[i][threadIdx.x] = rv;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int n = n0 + i, c = c0 + threadIdx.x;
+    if (n >= L) continue;
+    const long row = (long)b * L + n;
+    const float xv = tx[threadIdx.x][i];
+    if (lat) lat[row * C + c] = xv;
+    tok[row * 2 * C + c] = from_f<T>(xv);
+    tok[row * 2 * C + C + c] = from_f<T>(tr[threadIdx.x][i]);
+  }
+}
+
+// Euler step of the flow sampler, x <- x + (sigma' - sigma) v on unpinned tokens
+// (readings R12, R14), then the next patch-embed input for those channels.
+template <typename T>
+__global__ void euler_kernel(float* __restrict__ lat, const float* __restrict__ v, float dsig, int pinned_tokens,
+                             T* __restrict__ tok, int C, int L, long total) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+    const long row = i / C;
+    const int c = (int)(i % C);
+    const int n = (int)(row % L);
+    float x = lat[i];
+    if (n >= pinned_tokens) {
+      x = fmaf(dsig, v[i], x);
+      lat[i] = x;
+    }
+    tok[row * 2 * C + c] = from_f<T>(x);
+  }
+}
+
+__global__ void tokens_to_latent_kernel(const float* __restrict__ tok, float* __restrict__ out, int C, int L) {
+  __shared__ float t[32][33];
+  const int b = blockIdx.z;
+  const int n0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int n = n0 + i;
+    t[i][threadIdx.x] = n < L ? tok[((long)b * L + n) * C + c0 + threadIdx.x] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int c = c0 + i, n = n0 + threadIdx.x;
+    if (n < L) out[((long)b * C + c) * L + n] = t[threadIdx.x][i];
+  }
+}
+
+// ------------------------------------------------------------ seeded weights
+// SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) as a hash of a counter, two 53-bit
+// uniforms per element and one Box-Muller normal, all in float64 with explicitly
+// rounded operations so the value is the same as a host evaluation of the formula.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ double seeded_normal(uint64_t base, uint64_t i) {
+  const uint64_t c1 = base + 2ull * i;
+  const double u1 = (double)(splitmix64(c1) >> 11) * 0x1.0p-53;
+  const double u2 = (double)(splitmix64(c1 + 1ull) >> 11) * 0x1.0p-53;
+  const double r = sqrt(__dmul_rn(-2.0, log1p(-u1)));
+  const double a = __dmul_rn(2.0 * 3.141592653589793, u2);
+  return __dmul_rn(r, cos(a));
+}
+
+template <typename T>
+__global__ void gen_tensor_kernel(T* __restrict__ dst, long rows, long cols, long ld, uint64_t base, int kind,
+                                  double fan_sqrt, bool round_bf16) {
+  const long n = rows * cols;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
+    const double z = seeded_normal(base, (uint64_t)i);
+    double w;
+    if (kind == 0)
+      w = __ddiv_rn(z, fan_sqrt);
+    else if (kind == 1)
+      w = __dadd_rn(1.0, __dmul_rn(0.1, z));
+    else
+      w = __dmul_rn(0.1, z);
+    float f = __double2float_rn(w);
+    if (round_bf16) f = __bfloat162float(__float2bfloat16_rn(f));
+    dst[(i / cols) * ld + (i % cols)] = from_f<T>(f);
+  }
+}
+
+// rotary (cos, sin) per token and pair: pairs [0, pf) turn with the frame index,
+// [pf, pf+ph) with the row, the rest with the column; pair j of an axis with n dims
+// turns theta^(-2j/n) rad per position (reading R3; table shape as the `cos`/`sin`
+// fields of gizai:flashhead Types > FlashHead, one head's 64 columns).
+__global__ void rope_table_kernel(float2* tab, int F, int H, int W, int pf, int ph, int pw, double theta) {
+  const int L = F * H * W;
+  const int np = pf + ph + pw;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= L * np) return;
+  const int n = idx / np, d = idx % np;
+  const int f = n / (H * W), r = (n / W) % H, c = n % W;
+  int pos, j, ndim;
+  if (d < pf) {
+    pos = f; j = d; ndim = 2 * pf;
+  } else if (d < pf + ph) {
+    pos = r; j = d - pf; ndim = 2 * ph;
+  } else {
+    pos = c; j = d - pf - ph; ndim = 2 * pw;
+  }
+  const double ang = (double)pos * pow(theta, -2.0 * (double)j / (double)ndim);
+  tab[idx] = make_float2((float)cos(ang), (float)sin(ang));
+}
+
+__global__ void fill_kernel(float* p, long n, float v) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) p[i] = v;
+}
+
+// ------------------------------------------------------------ fp32 GEMM
+// 32 x 128 output tile per CTA; thread t owns row t%32 and the 32 columns (t/32)*32..
+// so the shared epilogue sees whole 32-column chunks of one row.
+template <int KIND>
+__global__ void __launch_bounds__(128) gemm_simt_kernel(const float* __restrict__ A, long lda,
+                                                        const float* __restrict__ W, long ldw, int M, int N, int K,
+                                                        EpiParams ep) {
+  __shared__ float As[32][33];
+  __shared__ float Ws[32][129];
+  __shared__ float ssq_s[4][32];
+  const int t = threadIdx.x;
+  const int r = t & 31, q = t >> 5;
+  const int m0 = blockIdx.y * 32, n0 = blockIdx.x * 128;
+  float acc[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    for (int i = t; i < 32 * 32; i += 128) {
+      const int kk = i & 31, rr = i >> 5;
+      As[kk][rr] = (m0 + rr < M && k0 + kk < K) ? A[(long)(m0 + rr) * lda + k0 + kk] : 0.f;
+    }
+    for (int i = t; i < 32 * 128; i += 128) {
+      const int kk = i & 31, cc = i >> 5;
+      Ws[kk][cc] = (k0 + kk < K) ? W[(long)(n0 + cc) * ldw + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < 32; ++kk) {
+      const float a = As[kk][r];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) acc[j] = fmaf(a, Ws[kk][q * 32 + j], acc[j]);
+    }
+    __syncthreads();
+  }
+  const int row = m0 + r;
+  float ssq = 0.f;
+  if (row < M) epi_chunk<KIND, float>(ep, row, n0 + q * 32, acc, ssq);
+  ssq_s[q][r] = ssq;
+  __syncthreads();
+  if (q == 0 && row < M) epi_group_end<KIND>(ep, row, n0, ssq_s[0][r] + ssq_s[1][r] + ssq_s[2][r] + ssq_s[3][r]);
+}
+
+inline int grid_for(long n, int block) {
+  long g = (n + block - 1) / block;
+  if (g > 148 * 16) g = 148 * 16;
+  return (int)(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+cudaError_t gemm_simt(const float* A, long lda, const float* W, long ldw, int M, int N, int K, int kind,
+                      const EpiParams& ep, cudaStream_t st) {
+  if (N % 128 != 0) return cudaErrorInvalidValue;
+  dim3 grid(N / 128, (M + 31) / 32);
+  switch (kind) {
+    case EPI_STORE: gemm_simt_kernel<EPI_STORE><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
+    case EPI_GELU: gemm_simt_kernel<EPI_GELU><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
+    case EPI_RESID: gemm_simt_kernel<EPI_RESID><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
+    case EPI_NORM: gemm_simt_kernel<EPI_NORM><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
+    case EPI_QKV: gemm_simt_kernel<EPI_QKV><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t cross_attn(const T* q, const float* ssq_q, const T* kv, long ldkv, int koff, int voff,
+                       const float* ssq_k, int ssq_k_ld, int ssq_k_off, int batch, int heads, int L, int F, int A,
+                       float eps, T* out, cudaStream_t st) {
+  if (A != 32) return cudaErrorInvalidValue;
+  dim3 grid(F, heads, batch);
+  cross_attn_kernel<T, 32><<<grid, 128, 0, st>>>(q, ssq_q, kv, ldkv, koff, voff, ssq_k, ssq_k_ld, ssq_k_off, heads,
+                                                 L, F, eps, 1.f / sqrtf(128.f), out);
+  return cudaGetLastError();
+}
+template cudaError_t cross_attn<float>(const float*, const float*, const float*, long, int, int, const float*, int,
+                                       int, int, int, int, int, int, float, float*, cudaStream_t);
+template cudaError_t cross_attn<bf16>(const bf16*, const float*, const bf16*, long, int, int, const float*, int,
+                                      int, int, int, int, int, int, float, bf16*, cudaStream_t);
+
+template <typename T>
+cudaError_t norm_rows(const float* x, T* out, int M, int D, int rows_per_batch, int mode, const float* shift,
+                      const float* scale, long mod_bstride, const float* w, const float* bb, float eps,
+                      cudaStream_t st) {
+  const int rows_per_cta = 8;
+  dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
+#define FH_NORM_CASE(NVV)                                                                                     \
+  case NVV:                                                                                                   \
+    norm_rows_kernel<T, NVV><<<grid, 32 * rows_per_cta, 0, st>>>(x, out, M, rows_per_batch, mode, shift, scale, \
+                                                                 mod_bstride, w, bb, eps);                    \
+    break;
+  switch (D / 128) {
+    FH_NORM_CASE(1) FH_NORM_CASE(2) FH_NORM_CASE(3) FH_NORM_CASE(4) FH_NORM_CASE(6) FH_NORM_CASE(8)
+    FH_NORM_CASE(12) FH_NORM_CASE(16)
+    default: return cudaErrorInvalidValue;
+  }
+#undef FH_NORM_CASE
+  return cudaGetLastError();
+}
+template cudaError_t norm_rows<float>(const float*, float*, int, int, int, int, const float*, const float*, long,
+                                      const float*, const float*, float, cudaStream_t);
+template cudaError_t norm_rows<bf16>(const float*, bf16*, int, int, int, int, const float*, const float*, long,
+                                     const float*, const float*, float, cudaStream_t);
+
+cudaError_t time_sinusoid(float* out, int batch, TVals tv, int dim, cudaStream_t st) {
+  const int n = batch * dim;
+  time_sinusoid_kernel<<<(n + 255) / 256, 256, 0, st>>>(out, batch, tv, dim);
+  return cudaGetLastError();
+}
+
+template <typename WT>
+cudaError_t gemv(const WT* W, const float* x, const float* bias, float* y, int N, int K, int batch, int silu_in,
+                 int silu_out, cudaStream_t st) {
+  if (batch > 8) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)batch * K * sizeof(float);
+  if (smem > 48 * 1024) return cudaErrorInvalidValue;
+  gemv_kernel<WT><<<(N + 7) / 8, 256, smem, st>>>(W, x, bias, y, N, K, batch, silu_in, silu_out);
+  return cudaGetLastError();
+}
+template cudaError_t gemv<float>(const float*, const float*, const float*, float*, int, int, int, int, int,
+                                 cudaStream_t);
+template cudaError_t gemv<bf16>(const bf16*, const float*, const float*, float*, int, int, int, int, int,
+                                cudaStream_t);
+
+cudaError_t assemble_mods(const float* table, const float* e0, const float* htable, const float* e, float* mods,
+                          float* hmods, int batch, int blocks, int D, cudaStream_t st) {
+  const long n = (long)batch * blocks * 6 * D + (long)batch * 2 * D;
+  assemble_mods_kernel<<<grid_for(n, 256), 256, 0, st>>>(table, e0, htable, e, mods, hmods, batch, blocks, D);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t prep_tokens(const float* x, const float* ref, const float* motion, int pin_frames, float* lat, T* tok,
+                        int batch, int C, int L, int HW, cudaStream_t st) {
+  if (C % 32 != 0) return cudaErrorInvalidValue;
+  dim3 grid((L + 31) / 32, C / 32, batch);
+  prep_tokens_kernel<T><<<grid, dim3(32, 8), 0, st>>>(x, ref, motion, pin_frames, lat, tok, C, L, HW);
+  return cudaGetLastError();
+}
+template cudaError_t prep_tokens<float>(const float*, const float*, const float*, int, float*, float*, int, int, int,
+                                        int, cudaStream_t);
+template cudaError_t prep_tokens<bf16>(const float*, const float*, const float*, int, float*, bf16*, int, int, int,
+                                       int, cudaStream_t);
+
+template <typename T>
+cudaError_t euler_step(float* lat, const float* v, float dsig, int pinned_tokens, T* tok, int batch, int C, int L,
+                       cudaStream_t st) {
+  const long n = (long)batch * L * C;
+  euler_kernel<T><<<grid_for(n, 256), 256, 0, st>>>(lat, v, dsig, pinned_tokens, tok, C, L, n);
+  return cudaGetLastError();
+}
+template cudaError_t euler_step<float>(float*, const float*, float, int, float*, int, int, int, cudaStream_t);
+template cudaError_t euler_step<bf16>(float*, const float*, float, int, bf16*, int, int, int, cudaStream_t);
+
+cudaError_t tokens_to_latent(const float* tok, float* out, int batch, int C, int L, cudaStream_t st) {
+  if (C % 32 != 0) return cudaErrorInvalidValue;
+  dim3 grid((L + 31) / 32, C / 32, batch);
+  tokens_to_latent_kernel<<<grid, dim3(32, 8), 0, st>>>(tok, out, C, L);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t gen_tensor(T* dst, long rows, long cols, long ld, uint64_t seed, int tid, int kind, int fan,
+                       bool round_bf16, cudaStream_t st) {
+  const uint64_t base = seed ^ ((uint64_t)tid << 40);
+  const long n = rows * cols;
+  gen_tensor_kernel<T><<<grid_for(n, 256), 256, 0, st>>>(dst, rows, cols, ld, base, kind, sqrt((double)fan),
+                                                         round_bf16);
+  return cudaGetLastError();
+}
+template cudaError_t gen_tensor<float>(float*, long, long, long, uint64_t, int, int, int, bool, cudaStream_t);
+template cudaError_t gen_tensor<bf16>(bf16*, long, long, long, uint64_t, int, int, int, bool, cudaStream_t);
+
+cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st) {
+  const int n = F * H * W * (pf + ph + pw);
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(tab, F, H, W, pf, ph, pw, (double)theta);
+  return cudaGetLastError();
+}
+
+cudaError_t fill_f32(float* p, long n, float v, cudaStream_t st) {
+  fill_kernel<<<grid_for(n, 256), 256, 0, st>>>(p, n, v);
+  return cudaGetLastError();
+}
+
+}  // namespace fh

@@ -20,13 +20,16 @@ from the same published definition; the GPU tests compare the two.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 MASK64 = (1 << 64) - 1
 GOLDEN_GAMMA = np.uint64(0x9E3779B97F4A7C15)
 _MIX1 = np.uint64(0xBF58476D1CE4E5B9)
 _MIX2 = np.uint64(0x94D049BB133111EB)
-_CHUNK = 1 << 22
+_CHUNK = 1 << 20
 
 
 def splitmix64(counter: np.ndarray) -> np.ndarray:
@@ -54,14 +57,32 @@ def _uniform_pair(seed: int, tid: int, start: int, n: int):
     return u1, u2
 
 
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(max_workers=max(1, min(32, len(os.sched_getaffinity(0)))))
+    return _POOL
+
+
 def normal(seed: int, tid: int, shape) -> np.ndarray:
     """float64 N(0,1) tensor of ``shape`` for tensor id ``tid``."""
     n = int(np.prod(shape, dtype=np.int64))
     out = np.empty(n, dtype=np.float64)
-    for s in range(0, n, _CHUNK):
+
+    def fill(s):
         m = min(_CHUNK, n - s)
         u1, u2 = _uniform_pair(seed, tid, s, m)
         out[s:s + m] = np.sqrt(-2.0 * np.log1p(-u1)) * np.cos(2.0 * np.pi * u2)
+
+    starts = range(0, n, _CHUNK)
+    if n > _CHUNK:
+        list(_pool().map(fill, starts))
+    else:
+        for s in starts:
+            fill(s)
     return out.reshape(shape)
 
 
