@@ -12,10 +12,11 @@
 //   warp 1     one thread issues tcgen05.mma: S_j = Q K_j^T into TMEM (double
 //              buffered), then O_j = P_j V_j into TMEM (double buffered; V is read
 //              MN-major straight from its [key][d] layout).
-//   warps 2-5  one query row per thread: S_j from TMEM, online softmax in base 2,
-//              P_j written as bf16 into 128-byte-swizzled shared memory for the
-//              next MMA, and O_j folded into a register accumulator that carries
-//              the running max correction.
+//   warps 2-9  two threads per query row (one per warpgroup, 64 keys and 64 output
+//              dims each): S_j from TMEM, online softmax in base 2, P_j written as
+//              bf16 into 128-byte-swizzled shared memory for the next MMA, and O_j
+//              folded into a register accumulator that carries the running max
+//              correction.
 //   The MMA thread issues S_{j+1} before P_j V_j so the tensor core works while the
 //   softmax warps exponentiate.
 // attn_simt_kernel (fp32 or bf16 inputs, CUDA cores): one query row per thread, a
@@ -29,6 +30,8 @@ namespace {
 
 constexpr int AT_BQ = 128;
 constexpr int AT_BK = 128;
+constexpr int AT_SOFTMAX_THREADS = 256;           // warps 2-9
+constexpr int AT_THREADS = 64 + AT_SOFTMAX_THREADS;
 constexpr uint32_t PANEL = 128 * 128;           // bytes of one [128 rows x 64 bf16] panel
 constexpr uint32_t TILE = 2 * PANEL;            // [128 rows x 128 bf16]
 // shared memory map (offsets from the 1024-aligned base)
@@ -37,7 +40,9 @@ constexpr uint32_t OFF_K = OFF_Q + TILE;        // 2 buffers
 constexpr uint32_t OFF_V = OFF_K + 2 * TILE;    // 2 buffers
 constexpr uint32_t OFF_P = OFF_V + 2 * TILE;    // 1 buffer
 constexpr uint32_t OFF_RK = OFF_P + TILE;       // float rk[2][128]
-constexpr uint32_t OFF_BAR = OFF_RK + 2 * 128 * 4;
+constexpr uint32_t OFF_MX = OFF_RK + 2 * 128 * 4;  // float [2][2][128] partial row maxima
+constexpr uint32_t OFF_LS = OFF_MX + 4 * 128 * 4;  // float [2][128] partial row sums
+constexpr uint32_t OFF_BAR = OFF_LS + 2 * 128 * 4;
 constexpr uint32_t AT_SMEM = OFF_BAR + 256 + 1024;
 
 __device__ __forceinline__ float ex2(float x) {
@@ -54,7 +59,7 @@ __device__ __forceinline__ float row_rms(const float* ssq, int ssq_ld, long row,
   return rsqrtf(s * inv_d + eps);
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(AT_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const float* __restrict__ ssq, int ssq_ld, int heads,
                    int L, float eps, float scale_log2, bf16* __restrict__ out, unsigned* err) {
@@ -74,7 +79,9 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* p_free = bars + 16;
   uint64_t* rk_full = bars + 17;  // [2]
   uint64_t* rk_free = bars + 19;  // [2]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 21);
+  uint64_t* mx_bar = bars + 21;   // [2]
+  uint64_t* l_bar = bars + 23;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -91,16 +98,18 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&s_free[i], AT_SOFTMAX_THREADS);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_free[i], 128);
+      mbar_init(&o_free[i], AT_SOFTMAX_THREADS);
     }
-    mbar_init(p_full, 128);
+    mbar_init(p_full, AT_SOFTMAX_THREADS);
     mbar_init(p_free, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&rk_full[i], 128);
-      mbar_init(&rk_free[i], 128);
+      mbar_init(&rk_full[i], AT_SOFTMAX_THREADS);
+      mbar_init(&rk_free[i], AT_SOFTMAX_THREADS);
+      mbar_init(&mx_bar[i], AT_SOFTMAX_THREADS);
     }
+    mbar_init(l_bar, AT_SOFTMAX_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -196,27 +205,31 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // softmax / correction / output: one query row per thread
-    const int quarter = warp & 3;
-    const int t = threadIdx.x - 64;  // 0..127 among the softmax threads
-    const int qi = qt * AT_BQ + quarter * 32 + lane;  // query index within the stream
+    // softmax / correction / output, warps 2-9: each query row belongs to one thread of each
+    // warpgroup; half 0 (warps 2-5) takes keys and output dims 0-63, half 1 (warps 6-9)
+    // takes 64-127. Only the partial row maxima cross between the halves (per tile, through
+    // shared memory and an mbarrier); the partial row sums are combined once at the end.
+    const int quarter = warp & 3;                      // TMEM lane quarter of this warp
+    const int half = (warp - 2) >> 2;
+    const int t = threadIdx.x - 64;                    // 0..255 among the softmax threads
+    const int rl = quarter * 32 + lane;                // row within the tile
+    const int qi = qt * AT_BQ + rl;                    // query index within the stream
     const bool qvalid = qi < L;
     const float inv_d = 1.f / (float)D;
     const float rq = row_rms(ssq, ssq_ld, (long)b * L + (qvalid ? qi : L - 1), 0, heads, inv_d, eps);
     const float qscale = rq * scale_log2;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint8_t* prow = smem + OFF_P + (uint32_t)(quarter * 32 + lane) * 128;
+    uint8_t* prow = smem + OFF_P + half * PANEL + (uint32_t)rl * 128;  // this half's 64 keys of P
     const int sw = lane & 7;  // (row % 8) for the 128-byte swizzle; quarter*32 is a multiple of 8
+    float* mxs = reinterpret_cast<float*>(smem + OFF_MX);  // [2 tiles][2 halves][128 rows]
+    float* lss = reinterpret_cast<float*>(smem + OFF_LS);  // [2 halves][128 rows]
 
     // per-key RMS factors of the K tiles, staged one tile ahead through two buffers
-    {
-      const int key = t;
-      rk_s[t] = key < L ? row_rms(ssq, ssq_ld, (long)b * L + key, heads, heads, inv_d, eps) : 0.f;
-      mbar_arrive(&rk_full[0]);
-    }
-    float o[128];
+    if (t < AT_BK) rk_s[t] = t < L ? row_rms(ssq, ssq_ld, (long)b * L + t, heads, heads, inv_d, eps) : 0.f;
+    mbar_arrive(&rk_full[0]);
+    float o[64];
 #pragma unroll
-    for (int d = 0; d < 128; ++d) o[d] = 0.f;
+    for (int d = 0; d < 64; ++d) o[d] = 0.f;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
 
@@ -229,25 +242,26 @@ __global__ void __launch_bounds__(192, 1)
           if (!ok) break;
         }
         const int key = (j + 1) * AT_BK + t;
-        rk_s[nb * 128 + t] = key < L ? row_rms(ssq, ssq_ld, (long)b * L + key, heads, heads, inv_d, eps) : 0.f;
+        if (t < AT_BK)
+          rk_s[nb * 128 + t] = key < L ? row_rms(ssq, ssq_ld, (long)b * L + key, heads, heads, inv_d, eps) : 0.f;
         mbar_arrive(&rk_full[nb]);
       }
       ok = mbar_wait(&rk_full[j & 1], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      const float* rk = rk_s + (j & 1) * 128;
+      const float* rk = rk_s + (j & 1) * 128 + half * 64;
       const int bf = j & 1;
       const uint32_t par = (j >> 1) & 1;
       ok = mbar_wait(&s_full[bf], par, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t s_t = tmem + lane_off + bf * 128;
-      const int kvalid = L - j * AT_BK;  // keys of this tile that exist
-      // pass 1: row max
+      const uint32_t s_t = tmem + lane_off + bf * 128 + half * 64;
+      const int kvalid = L - j * AT_BK - half * 64;  // keys of this half-tile that exist
+      // pass 1: partial row max over this half's keys, then exchange with the other half
       float mx = -INFINITY;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         float v[32];
         tmem_ld32(s_t + c, v);
         tc_wait_ld();
@@ -255,6 +269,13 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = 0; e < 32; ++e)
           if (c + e < kvalid) mx = fmaxf(mx, v[e] * rk[c + e]);
       }
+      float* mxt = mxs + (j & 1) * 256;
+      mxt[half * 128 + rl] = mx;
+      mbar_arrive(&mx_bar[j & 1]);
+      ok = mbar_wait(&mx_bar[j & 1], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      mx = fmaxf(mx, mxt[(1 - half) * 128 + rl]);
       const float m_new = fmaxf(m_run, mx * qscale);
       const float alpha = ex2(m_run - m_new);
       // P_j overwrites the P buffer: wait until P_{j-1} V_{j-1} has consumed it
@@ -263,10 +284,10 @@ __global__ void __launch_bounds__(192, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
-      // pass 2: probabilities, row sum, bf16 P into swizzled shared memory
+      // pass 2: probabilities, partial row sum, bf16 P into this half's swizzled panel
       float rs = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         float v[32];
         tmem_ld32(s_t + c, v);
         tc_wait_ld();
@@ -276,14 +297,13 @@ __global__ void __launch_bounds__(192, 1)
           v[e] = p;
           rs += p;
         }
-        uint8_t* panel = prow + (c >> 6) * PANEL;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const int chunk = ((c & 63) >> 3) + q;
+          const int chunk = (c >> 3) + q;
           __nv_bfloat162 hv[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) hv[u] = __floats2bfloat162_rn(v[q * 8 + 2 * u], v[q * 8 + 2 * u + 1]);
-          *reinterpret_cast<uint4*>(panel + ((chunk ^ sw) << 4)) = *reinterpret_cast<uint4*>(hv);
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ sw) << 4)) = *reinterpret_cast<uint4*>(hv);
         }
       }
       mbar_arrive(&rk_free[bf]);
@@ -293,16 +313,16 @@ __global__ void __launch_bounds__(192, 1)
       mbar_arrive(p_full);
       l_run = l_run * alpha + rs;
       m_run = m_new;
-      // fold O_{j-1} (relative to the previous max) and rescale to the new max
+      // fold this half's 64 dims of O_{j-1} (relative to the previous max), rescale to the new max
       if (j >= 1) {
         const int pb = (j - 1) & 1;
         ok = mbar_wait(&o_full[pb], ((j - 1) >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t o_t = tmem + lane_off + 256 + pb * 128;
+        const uint32_t o_t = tmem + lane_off + 256 + pb * 128 + half * 64;
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = 0; c < 64; c += 32) {
           float v[32];
           tmem_ld32(o_t + c, v);
           tc_wait_ld();
@@ -319,20 +339,25 @@ __global__ void __launch_bounds__(192, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        const uint32_t o_t = tmem + lane_off + 256 + pb * 128;
+        const uint32_t o_t = tmem + lane_off + 256 + pb * 128 + half * 64;
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = 0; c < 64; c += 32) {
           float v[32];
           tmem_ld32(o_t + c, v);
           tc_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[c + e] += v[e];
         }
-        const float inv_l = 1.f / l_run;
-        if (qvalid) {
-          bf16* dst = out + ((long)b * L + qi) * D + h * 128;
+        // the row's normaliser is the sum of both halves' partial sums
+        lss[half * 128 + rl] = l_run;
+        mbar_arrive(l_bar);
+        ok = mbar_wait(l_bar, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok && qvalid) {
+          const float inv_l = 1.f / (l_run + lss[(1 - half) * 128 + rl]);
+          bf16* dst = out + ((long)b * L + qi) * D + h * 128 + half * 64;
 #pragma unroll
-          for (int d = 0; d < 128; d += 8) {
+          for (int d = 0; d < 64; d += 8) {
             float w[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) w[e] = o[d + e] * inv_l;
@@ -436,7 +461,7 @@ cudaError_t attn_tc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMa
                     cudaStream_t st) {
   const float scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   dim3 grid((L + AT_BQ - 1) / AT_BQ, heads, batch);
-  attn_tc_kernel<<<grid, 192, AT_SMEM, st>>>(q, k, v, ssq, ssq_ld, heads, L, eps, scale_log2, out, err);
+  attn_tc_kernel<<<grid, AT_THREADS, AT_SMEM, st>>>(q, k, v, ssq, ssq_ld, heads, L, eps, scale_log2, out, err);
   return cudaGetLastError();
 }
 

@@ -82,82 +82,102 @@ __global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ ou
 }
 
 // ------------------------------------------------------ per-frame cross-attention
-// A token of latent frame f attends to frame f's A audio tokens only (gizai:flashhead,
-// opening paragraph: 5 latent frames of 32 audio tokens; reading R5). One CTA per
-// (frame, head, stream) stages that frame's keys/values (fp32) and key RMS factors in
-// shared memory; one query per thread.
-template <typename T, int A>
-__global__ void __launch_bounds__(128) cross_attn_kernel(const T* __restrict__ q, const float* __restrict__ ssq_q,
-                                                         const T* __restrict__ kv, long ldkv, int koff, int voff,
-                                                         const float* __restrict__ ssq_k, int ssq_k_ld,
-                                                         int ssq_k_off, int heads, int L, int F, float eps,
-                                                         float scale, T* __restrict__ out) {
+// A token of latent frame f attends to frame f's A = 32 audio tokens only (gizai:flashhead,
+// opening paragraph: 5 latent frames of 32 audio tokens; reading R5). One CTA per (frame,
+// head, stream, chunk of XA_QPB queries) stages that frame's keys/values (fp32) and key RMS
+// factors in shared memory. One warp per query: lane a scores audio key a, the softmax is a
+// pair of warp reductions, and lane l accumulates output dims 4l..4l+3.
+constexpr int XA_WARPS = 8;
+constexpr int XA_QPW = 8;                    // queries per warp
+constexpr int XA_QPB = XA_WARPS * XA_QPW;    // queries per CTA
+
+template <typename T>
+__global__ void __launch_bounds__(XA_WARPS * 32)
+    cross_attn_kernel(const T* __restrict__ q, const float* __restrict__ ssq_q, const T* __restrict__ kv, long ldkv,
+                      int koff, int voff, const float* __restrict__ ssq_k, int ssq_k_ld, int ssq_k_off, int heads,
+                      int L, int F, int nqc, float eps, float scale, T* __restrict__ out) {
+  constexpr int A = 32;
   __shared__ float ks[A][129];
-  __shared__ float vs[A][128];
+  __shared__ __align__(16) float vs[A][128];
   __shared__ float rks[A];
-  const int f = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  __shared__ float qs[XA_WARPS][128];
+  const int f = blockIdx.x / nqc, qc = blockIdx.x % nqc;
+  const int h = blockIdx.y, b = blockIdx.z;
   const int D = heads * 128;
   const float inv_d = 1.f / (float)D;
   const long kv_row0 = ((long)b * F + f) * A;
-  for (int idx = threadIdx.x; idx < A * 128; idx += blockDim.x) {
-    const int a = idx >> 7, d = idx & 127;
+  for (int idx = threadIdx.x; idx < A * 16; idx += blockDim.x) {
+    const int a = idx >> 4, d = (idx & 15) * 8;
     const T* r = kv + (kv_row0 + a) * ldkv;
-    ks[a][d] = to_f(r[koff + h * 128 + d]);
-    vs[a][d] = to_f(r[voff + h * 128 + d]);
+    float tk[8], tv[8];
+    load8(r + koff + h * 128 + d, tk);
+    load8(r + voff + h * 128 + d, tv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      ks[a][d + e] = tk[e];
+      vs[a][d + e] = tv[e];
+    }
   }
-  for (int a = threadIdx.x; a < A; a += blockDim.x) {
-    const float* p = ssq_k + (kv_row0 + a) * ssq_k_ld + ssq_k_off;
+  if (threadIdx.x < A) {
+    const float* p = ssq_k + (kv_row0 + threadIdx.x) * ssq_k_ld + ssq_k_off;
     float s = 0.f;
     for (int i = 0; i < heads; ++i) s += p[i];
-    rks[a] = rsqrtf(s * inv_d + eps);
+    rks[threadIdx.x] = rsqrtf(s * inv_d + eps);
   }
   __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int HW = L / F;
-  for (int n = threadIdx.x; n < HW; n += blockDim.x) {
+  const float rk = rks[lane] * scale;
+  for (int i = 0; i < XA_QPW; ++i) {
+    const int n = qc * XA_QPB + warp * XA_QPW + i;
+    if (n >= HW) break;
     const long row = (long)b * L + (long)f * HW + n;
-    const float* pq = ssq_q + row * heads;
-    float sq = 0.f;
-    for (int i = 0; i < heads; ++i) sq += pq[i];
-    const float rq = rsqrtf(sq * inv_d + eps) * scale;
-    const T* qr = q + row * D + h * 128;
-    float s[A];
-#pragma unroll
-    for (int a = 0; a < A; ++a) s[a] = 0.f;
-#pragma unroll 1
-    for (int d0 = 0; d0 < 128; d0 += 8) {
-      float qv[8];
-      load8(qr + d0, qv);
-#pragma unroll
-      for (int a = 0; a < A; ++a) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s[a] = fmaf(qv[e], ks[a][d0 + e], s[a]);
-      }
+    // query slice and RMS factor
+    float sq = lane < heads ? ssq_q[row * heads + lane] : 0.f;
+    sq = warp_sum(sq);
+    const float rq = rsqrtf(sq * inv_d + eps);
+    const T* qr = q + row * D + h * 128 + lane * 4;
+    float4 qv;
+    if constexpr (sizeof(T) == 2) {
+      uint2 u = *reinterpret_cast<const uint2*>(qr);
+      float2 a0 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+      float2 a1 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+      qv = make_float4(a0.x, a0.y, a1.x, a1.y);
+    } else {
+      qv = *reinterpret_cast<const float4*>(qr);
     }
-    float m = -INFINITY;
-#pragma unroll
+    __syncwarp();
+    *reinterpret_cast<float4*>(&qs[warp][lane * 4]) = qv;
+    __syncwarp();
+    // lane = audio key
+    float s = 0.f;
+#pragma unroll 16
+    for (int d = 0; d < 128; ++d) s = fmaf(qs[warp][d], ks[lane][d], s);
+    s *= rq * rk;
+    const float m = warp_max(s);
+    const float p = expf(s - m);
+    const float inv_z = 1.f / warp_sum(p);
+    // lane = 4 output dims
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
     for (int a = 0; a < A; ++a) {
-      s[a] *= rq * rks[a];
-      m = fmaxf(m, s[a]);
+      const float pa = __shfl_sync(0xffffffffu, p, a);
+      const float4 vv = *reinterpret_cast<const float4*>(&vs[a][lane * 4]);
+      o.x = fmaf(pa, vv.x, o.x);
+      o.y = fmaf(pa, vv.y, o.y);
+      o.z = fmaf(pa, vv.z, o.z);
+      o.w = fmaf(pa, vv.w, o.w);
     }
-    float z = 0.f;
-#pragma unroll
-    for (int a = 0; a < A; ++a) {
-      s[a] = expf(s[a] - m);
-      z += s[a];
-    }
-    const float iz = 1.f / z;
-    T* orow = out + row * D + h * 128;
-#pragma unroll 1
-    for (int d0 = 0; d0 < 128; d0 += 8) {
-      float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int a = 0; a < A; ++a) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = fmaf(s[a], vs[a][d0 + e], o[e]);
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] *= iz;
-      store8(orow + d0, o);
+    T* dst = out + row * D + h * 128 + lane * 4;
+    if constexpr (sizeof(T) == 2) {
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(o.x * inv_z, o.y * inv_z);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(o.z * inv_z, o.w * inv_z);
+      uint2 u;
+      u.x = *reinterpret_cast<uint32_t*>(&h0);
+      u.y = *reinterpret_cast<uint32_t*>(&h1);
+      *reinterpret_cast<uint2*>(dst) = u;
+    } else {
+      *reinterpret_cast<float4*>(dst) = make_float4(o.x * inv_z, o.y * inv_z, o.z * inv_z, o.w * inv_z);
     }
   }
 }
@@ -431,10 +451,12 @@ template <typename T>
 cudaError_t cross_attn(const T* q, const float* ssq_q, const T* kv, long ldkv, int koff, int voff,
                        const float* ssq_k, int ssq_k_ld, int ssq_k_off, int batch, int heads, int L, int F, int A,
                        float eps, T* out, cudaStream_t st) {
-  if (A != 32) return cudaErrorInvalidValue;
-  dim3 grid(F, heads, batch);
-  cross_attn_kernel<T, 32><<<grid, 128, 0, st>>>(q, ssq_q, kv, ldkv, koff, voff, ssq_k, ssq_k_ld, ssq_k_off, heads,
-                                                 L, F, eps, 1.f / sqrtf(128.f), out);
+  if (A != 32 || heads > 32) return cudaErrorInvalidValue;
+  const int HW = L / F;
+  const int nqc = (HW + XA_QPB - 1) / XA_QPB;
+  dim3 grid(F * nqc, heads, batch);
+  cross_attn_kernel<T><<<grid, XA_WARPS * 32, 0, st>>>(q, ssq_q, kv, ldkv, koff, voff, ssq_k, ssq_k_ld, ssq_k_off,
+                                                      heads, L, F, nqc, eps, 1.f / sqrtf(128.f), out);
   return cudaGetLastError();
 }
 template cudaError_t cross_attn<float>(const float*, const float*, const float*, long, int, int, const float*, int,
