@@ -105,6 +105,7 @@ def load_library() -> ctypes.CDLL:
         "fh_dit_get_timing": (I, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I)]),
         "fh_last_error": (ctypes.c_char_p, []),
         "fh_op_linear": (I, [P, P, P, P, I, I, I, I, P]),
+        "fh_dit_block_forward_noalloc": (I, [P, I, P, P, P, P, I, P]),
         "fh_op_attention": (I, [P, P, P, P, P, I, I, I, F, I, P]),
     }
     for name, (res, args) in sig.items():
@@ -187,6 +188,15 @@ class DiT:
         out = torch.empty_like(x) if out is None else out
         _check(load_library().fh_dit_block_forward(self._h, block, _ptr(x), _ptr(out), _ptr(audio), _farr(t), B,
                                                    _ptr(ws), _stream(stream)))
+        return out
+
+    def block_forward_noalloc(self, block: int, x, audio, t, out=None, stream=None):
+        """block_forward on the library's static scratch (no workspace, no allocation by the library)."""
+        import torch
+        B = x.shape[0]
+        out = torch.empty_like(x) if out is None else out
+        _check(load_library().fh_dit_block_forward_noalloc(self._h, block, _ptr(x), _ptr(out), _ptr(audio),
+                                                           _farr(t), B, _stream(stream)))
         return out
 
     def predict_flow(self, x_noisy, ref, audio, sigma: float, ws, out=None, stream=None):

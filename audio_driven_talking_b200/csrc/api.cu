@@ -1031,3 +1031,9 @@ int fh_op_attention(const void* q, const void* k, const void* v, const float* ss
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ internal helpers for other files
+namespace fh {
+int set_error(int code, const char* msg) { return fail(code, "%s", msg); }
+int model_device(const fh_dit* m) { return m ? m->device : -1; }
+}  // namespace fh

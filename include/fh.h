@@ -172,6 +172,24 @@ int fh_dit_last_launch_count(const fh_dit* m);
 int fh_dit_set_timing(fh_dit* m, int kernel_class);
 int fh_dit_get_timing(fh_dit* m, double* mean_us, int* launches);
 
+/* fh_dit_block_forward without a workspace argument, for callers that cannot allocate
+ * device memory where they run a block (code running while a stream is captured into a
+ * CUDA graph, plugins inside a framework that owns all device memory, real-time threads
+ * that must not take allocator locks). The pages have no counterpart: this is a
+ * deployment variant, not a step of the method. The scratch is a file-scope __device__
+ * array of FH_STATIC_SCRATCH_BYTES (16 MiB) inside the library, held on every GPU that
+ * loads the library until the process exits; calls whose fh_dit_workspace_bytes exceeds
+ * it fail with FH_ERR_SHAPE (the full 1536-wide network needs more: use
+ * fh_dit_block_forward there). The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, which may load the library's module): make that first
+ * call before any stream capture. Every call on a device shares the one array and it
+ * keeps the last call's contents; calls that overlap in time on the GPU (different
+ * streams, or different handles) race on it. Nothing in it needs to start at zero.
+ * Arguments and errors otherwise as fh_dit_block_forward. Allocates nothing. */
+#define FH_STATIC_SCRATCH_BYTES (16u << 20)
+int fh_dit_block_forward_noalloc(fh_dit* m, int block, const float* x_in, float* x_out, const void* audio,
+                                 const float* t, int batch, void* stream);
+
 /* Thread-local text of the last error ("" if none). */
 const char* fh_last_error(void);
 
