@@ -124,6 +124,8 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  pdl_launch_dependents();
+  pdl_wait();  // q, k, v and the sums of squares come from the preceding QKV projection
 
   if (warp == 0) {
     if (lane == 0) {
@@ -384,6 +386,8 @@ __global__ void __launch_bounds__(64) attn_simt_kernel(const T* __restrict__ Q, 
                                                        const T* __restrict__ V, const float* __restrict__ ssq,
                                                        int ssq_ld, int heads, int L, float eps, float scale,
                                                        T* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float ks[SA_KC][128];
   __shared__ float vs[SA_KC][128];
   __shared__ float rks[SA_KC];
@@ -461,7 +465,7 @@ cudaError_t attn_tc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMa
                     cudaStream_t st) {
   const float scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   dim3 grid((L + AT_BQ - 1) / AT_BQ, heads, batch);
-  attn_tc_kernel<<<grid, AT_THREADS, AT_SMEM, st>>>(q, k, v, ssq, ssq_ld, heads, L, eps, scale_log2, out, err);
+  { cudaError_t e_ = launch_pdl(attn_tc_kernel, dim3(grid), dim3(AT_THREADS), AT_SMEM, st, q, k, v, ssq, ssq_ld, heads, L, eps, scale_log2, out, err); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 
@@ -469,7 +473,7 @@ template <typename T>
 cudaError_t attn_simt(const T* q, const T* k, const T* v, const float* ssq, int ssq_ld, int batch, int heads, int L,
                       float eps, T* out, cudaStream_t st) {
   dim3 grid((L + 63) / 64, heads, batch);
-  attn_simt_kernel<T><<<grid, 64, 0, st>>>(q, k, v, ssq, ssq_ld, heads, L, eps, 1.f / sqrtf(128.f), out);
+  { cudaError_t e_ = launch_pdl(attn_simt_kernel<T>, dim3(grid), dim3(64), 0, st, q, k, v, ssq, ssq_ld, heads, L, eps, 1.f / sqrtf(128.f), out); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 

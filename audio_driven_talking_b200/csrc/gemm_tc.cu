@@ -92,20 +92,36 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
+  pdl_launch_dependents();
   if (warp == 0) {
     if (lane == 0) {
+      // The weights W are never written by any kernel: start streaming the first stages'
+      // W tiles before waiting for the kernels this one depends on (programmatic launch).
+      int pre = 0;
+      if ((int)blockIdx.x < ntiles) {
+        const int n0 = ((int)blockIdx.x / num_m) * BN;
+        pre = nk < S::STAGES ? nk : S::STAGES;
+        for (int s = 0; s < pre; ++s) {
+          mbar_expect_tx(&full[s], S::STAGE_BYTES);
+          tma_load_2d(&tmB, &full[s], smem + s * S::STAGE_BYTES + S::A_BYTES, s * BK, n0);
+        }
+      }
+      pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
       long issues = 0;
-      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+      bool first = true;
+      for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, first = false) {
         const int m0 = (tile % num_m) * BM;
         const int n0 = (tile / num_m) * BN;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) goto producer_done;
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
-          mbar_expect_tx(&full[stage], S::STAGE_BYTES);
+          if (!(first && kb < pre)) {
+            mbar_expect_tx(&full[stage], S::STAGE_BYTES);
+            tma_load_2d(&tmB, &full[stage], sa + S::A_BYTES, kb * BK, n0);
+          }
           tma_load_2d(&tmA, &full[stage], sa, kb * BK, m0);
-          tma_load_2d(&tmB, &full[stage], sa + S::A_BYTES, kb * BK, n0);
           ++issues;
           if (++stage == S::STAGES) {
             stage = 0;
@@ -115,7 +131,10 @@ __global__ void __launch_bounds__(192, 1)
       }
     producer_done:
       if (*abort_flag) {
-        // let every copy this thread started land before the CTA's shared memory goes away
+        // let every copy this thread started land before the CTA's shared memory goes away;
+        // W tiles issued ahead of the dependency wait whose A half never followed cannot
+        // complete their barrier phase, so their wait simply runs out its bounded time
+        for (long s = issues; s < pre; ++s) drain_wait(&full[s], 0);
         for (int s = 0; s < S::STAGES; ++s) {
           if (issues <= 0) break;
           int st = stage - 1 - s;
@@ -167,6 +186,7 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    pdl_wait();                    // the epilogue reads and writes global memory
     int local = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
@@ -209,8 +229,7 @@ cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, 
   using S = TcShape<BN>;
   const int tiles = ((M + BM - 1) / BM) * (N / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_tc_kernel<BN, KIND, OutT><<<grid, 192, S::SMEM, st>>>(a, b, M, N, K, ep, err);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<BN, KIND, OutT>, dim3(grid), dim3(192), S::SMEM, st, a, b, M, N, K, ep, err);
 }
 
 template <int BN, int KIND, typename OutT>

@@ -22,6 +22,8 @@ __global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ ou
                                  int mode, const float* __restrict__ shift, const float* __restrict__ scale,
                                  long mod_bstride, const float* __restrict__ w, const float* __restrict__ bb,
                                  float eps) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int D = NV * 128;
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -96,6 +98,8 @@ __global__ void __launch_bounds__(XA_WARPS * 32)
     cross_attn_kernel(const T* __restrict__ q, const float* __restrict__ ssq_q, const T* __restrict__ kv, long ldkv,
                       int koff, int voff, const float* __restrict__ ssq_k, int ssq_k_ld, int ssq_k_off, int heads,
                       int L, int F, int nqc, float eps, float scale, T* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   constexpr int A = 32;
   __shared__ float ks[A][129];
   __shared__ __align__(16) float vs[A][128];
@@ -106,6 +110,27 @@ __global__ void __launch_bounds__(XA_WARPS * 32)
   const int D = heads * 128;
   const float inv_d = 1.f / (float)D;
   const long kv_row0 = ((long)b * F + f) * A;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int HW = L / F;
+  // issue every global load of this warp's queries up front (they are independent)
+  const int n0 = qc * XA_QPB + warp * XA_QPW;
+  float4 qpre[XA_QPW];
+  float sqpre[XA_QPW];
+#pragma unroll
+  for (int i = 0; i < XA_QPW; ++i) {
+    const int n = n0 + i < HW ? n0 + i : HW - 1;
+    const long row = (long)b * L + (long)f * HW + n;
+    sqpre[i] = lane < heads ? ssq_q[row * heads + lane] : 0.f;
+    const T* qr = q + row * D + h * 128 + lane * 4;
+    if constexpr (sizeof(T) == 2) {
+      uint2 u = *reinterpret_cast<const uint2*>(qr);
+      float2 a0 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+      float2 a1 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+      qpre[i] = make_float4(a0.x, a0.y, a1.x, a1.y);
+    } else {
+      qpre[i] = *reinterpret_cast<const float4*>(qr);
+    }
+  }
   for (int idx = threadIdx.x; idx < A * 16; idx += blockDim.x) {
     const int a = idx >> 4, d = (idx & 15) * 8;
     const T* r = kv + (kv_row0 + a) * ldkv;
@@ -125,27 +150,14 @@ __global__ void __launch_bounds__(XA_WARPS * 32)
     rks[threadIdx.x] = rsqrtf(s * inv_d + eps);
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int HW = L / F;
   const float rk = rks[lane] * scale;
+#pragma unroll
   for (int i = 0; i < XA_QPW; ++i) {
-    const int n = qc * XA_QPB + warp * XA_QPW + i;
+    const int n = n0 + i;
     if (n >= HW) break;
     const long row = (long)b * L + (long)f * HW + n;
-    // query slice and RMS factor
-    float sq = lane < heads ? ssq_q[row * heads + lane] : 0.f;
-    sq = warp_sum(sq);
-    const float rq = rsqrtf(sq * inv_d + eps);
-    const T* qr = q + row * D + h * 128 + lane * 4;
-    float4 qv;
-    if constexpr (sizeof(T) == 2) {
-      uint2 u = *reinterpret_cast<const uint2*>(qr);
-      float2 a0 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
-      float2 a1 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
-      qv = make_float4(a0.x, a0.y, a1.x, a1.y);
-    } else {
-      qv = *reinterpret_cast<const float4*>(qr);
-    }
+    const float rq = rsqrtf(warp_sum(sqpre[i]) * inv_d + eps);
+    const float4 qv = qpre[i];
     __syncwarp();
     *reinterpret_cast<float4*>(&qs[warp][lane * 4]) = qv;
     __syncwarp();
@@ -187,6 +199,8 @@ __global__ void __launch_bounds__(XA_WARPS * 32)
 // (reading R10 of the timestep embedding that yields the per-step modulations,
 // gizai:flashhead Types > FlashHead, field headMods).
 __global__ void time_sinusoid_kernel(float* out, int batch, TVals tv, int dim) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int half = dim / 2;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= batch * dim) return;
@@ -201,6 +215,8 @@ __global__ void time_sinusoid_kernel(float* out, int batch, TVals tv, int dim) {
 template <typename WT>
 __global__ void gemv_kernel(const WT* __restrict__ W, const float* __restrict__ x, const float* __restrict__ bias,
                             float* __restrict__ y, int N, int K, int batch, int silu_in, int silu_out) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ float xs[];
   for (int i = threadIdx.x; i < batch * K; i += blockDim.x) {
     const float v = x[i];
@@ -230,6 +246,8 @@ __global__ void assemble_mods_kernel(const float* __restrict__ table, const floa
                                      const float* __restrict__ htable, const float* __restrict__ e,
                                      float* __restrict__ mods, float* __restrict__ hmods, int batch, int blocks,
                                      int D) {
+  pdl_launch_dependents();
+  pdl_wait();
   const long per = (long)blocks * 6 * D;
   const long total = (long)batch * per;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total + (long)batch * 2 * D;
@@ -254,6 +272,8 @@ template <typename T>
 __global__ void prep_tokens_kernel(const float* __restrict__ x, const float* __restrict__ ref,
                                    const float* __restrict__ motion, int pin_frames, float* __restrict__ lat,
                                    T* __restrict__ tok, int C, int L, int HW) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float tx[32][33];
   __shared__ float tr[32][33];
   const int b = blockIdx.z;
@@ -287,6 +307,8 @@ __global__ void prep_tokens_kernel(const float* __restrict__ x, const float* __r
 template <typename T>
 __global__ void euler_kernel(float* __restrict__ lat, const float* __restrict__ v, float dsig, int pinned_tokens,
                              T* __restrict__ tok, int C, int L, long total) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
     const long row = i / C;
     const int c = (int)(i % C);
@@ -301,6 +323,8 @@ __global__ void euler_kernel(float* __restrict__ lat, const float* __restrict__ 
 }
 
 __global__ void tokens_to_latent_kernel(const float* __restrict__ tok, float* __restrict__ out, int C, int L) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float t[32][33];
   const int b = blockIdx.z;
   const int n0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
@@ -338,6 +362,8 @@ __device__ __forceinline__ double seeded_normal(uint64_t base, uint64_t i) {
 template <typename T>
 __global__ void gen_tensor_kernel(T* __restrict__ dst, long rows, long cols, long ld, uint64_t base, int kind,
                                   double fan_sqrt, bool round_bf16) {
+  pdl_launch_dependents();
+  pdl_wait();
   const long n = rows * cols;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) {
     const double z = seeded_normal(base, (uint64_t)i);
@@ -359,6 +385,8 @@ __global__ void gen_tensor_kernel(T* __restrict__ dst, long rows, long cols, lon
 // turns theta^(-2j/n) rad per position (reading R3; table shape as the `cos`/`sin`
 // fields of gizai:flashhead Types > FlashHead, one head's 64 columns).
 __global__ void rope_table_kernel(float2* tab, int F, int H, int W, int pf, int ph, int pw, double theta) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int L = F * H * W;
   const int np = pf + ph + pw;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -378,6 +406,8 @@ __global__ void rope_table_kernel(float2* tab, int F, int H, int W, int pf, int 
 }
 
 __global__ void fill_kernel(float* p, long n, float v) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x) p[i] = v;
 }
 
@@ -388,6 +418,8 @@ template <int KIND>
 __global__ void __launch_bounds__(128) gemm_simt_kernel(const float* __restrict__ A, long lda,
                                                         const float* __restrict__ W, long ldw, int M, int N, int K,
                                                         EpiParams ep) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float As[32][33];
   __shared__ float Ws[32][129];
   __shared__ float ssq_s[4][32];
@@ -437,11 +469,11 @@ cudaError_t gemm_simt(const float* A, long lda, const float* W, long ldw, int M,
   if (N % 128 != 0) return cudaErrorInvalidValue;
   dim3 grid(N / 128, (M + 31) / 32);
   switch (kind) {
-    case EPI_STORE: gemm_simt_kernel<EPI_STORE><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
-    case EPI_GELU: gemm_simt_kernel<EPI_GELU><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
-    case EPI_RESID: gemm_simt_kernel<EPI_RESID><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
-    case EPI_NORM: gemm_simt_kernel<EPI_NORM><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
-    case EPI_QKV: gemm_simt_kernel<EPI_QKV><<<grid, 128, 0, st>>>(A, lda, W, ldw, M, N, K, ep); break;
+    case EPI_STORE: { cudaError_t e_ = launch_pdl(gemm_simt_kernel<EPI_STORE>, dim3(grid), dim3(128), 0, st, A, lda, W, ldw, M, N, K, ep); if (e_ != cudaSuccess) return e_; } break;
+    case EPI_GELU: { cudaError_t e_ = launch_pdl(gemm_simt_kernel<EPI_GELU>, dim3(grid), dim3(128), 0, st, A, lda, W, ldw, M, N, K, ep); if (e_ != cudaSuccess) return e_; } break;
+    case EPI_RESID: { cudaError_t e_ = launch_pdl(gemm_simt_kernel<EPI_RESID>, dim3(grid), dim3(128), 0, st, A, lda, W, ldw, M, N, K, ep); if (e_ != cudaSuccess) return e_; } break;
+    case EPI_NORM: { cudaError_t e_ = launch_pdl(gemm_simt_kernel<EPI_NORM>, dim3(grid), dim3(128), 0, st, A, lda, W, ldw, M, N, K, ep); if (e_ != cudaSuccess) return e_; } break;
+    case EPI_QKV: { cudaError_t e_ = launch_pdl(gemm_simt_kernel<EPI_QKV>, dim3(grid), dim3(128), 0, st, A, lda, W, ldw, M, N, K, ep); if (e_ != cudaSuccess) return e_; } break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -455,8 +487,8 @@ cudaError_t cross_attn(const T* q, const float* ssq_q, const T* kv, long ldkv, i
   const int HW = L / F;
   const int nqc = (HW + XA_QPB - 1) / XA_QPB;
   dim3 grid(F * nqc, heads, batch);
-  cross_attn_kernel<T><<<grid, XA_WARPS * 32, 0, st>>>(q, ssq_q, kv, ldkv, koff, voff, ssq_k, ssq_k_ld, ssq_k_off,
-                                                      heads, L, F, nqc, eps, 1.f / sqrtf(128.f), out);
+  { cudaError_t e_ = launch_pdl(cross_attn_kernel<T>, dim3(grid), dim3(XA_WARPS * 32), 0, st, q, ssq_q, kv, ldkv, koff, voff, ssq_k, ssq_k_ld, ssq_k_off,
+                                                      heads, L, F, nqc, eps, 1.f / sqrtf(128.f), out); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 template cudaError_t cross_attn<float>(const float*, const float*, const float*, long, int, int, const float*, int,
@@ -472,8 +504,8 @@ cudaError_t norm_rows(const float* x, T* out, int M, int D, int rows_per_batch, 
   dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
 #define FH_NORM_CASE(NVV)                                                                                     \
   case NVV:                                                                                                   \
-    norm_rows_kernel<T, NVV><<<grid, 32 * rows_per_cta, 0, st>>>(x, out, M, rows_per_batch, mode, shift, scale, \
-                                                                 mod_bstride, w, bb, eps);                    \
+    { cudaError_t e_ = launch_pdl(norm_rows_kernel<T, NVV>, dim3(grid), dim3(32 * rows_per_cta), 0, st, x, out, M, rows_per_batch, mode, shift, scale, \
+                                                                 mod_bstride, w, bb, eps); if (e_ != cudaSuccess) return e_; }                    \
     break;
   switch (D / 128) {
     FH_NORM_CASE(1) FH_NORM_CASE(2) FH_NORM_CASE(3) FH_NORM_CASE(4) FH_NORM_CASE(6) FH_NORM_CASE(8)
@@ -490,7 +522,7 @@ template cudaError_t norm_rows<bf16>(const float*, bf16*, int, int, int, int, co
 
 cudaError_t time_sinusoid(float* out, int batch, TVals tv, int dim, cudaStream_t st) {
   const int n = batch * dim;
-  time_sinusoid_kernel<<<(n + 255) / 256, 256, 0, st>>>(out, batch, tv, dim);
+  { cudaError_t e_ = launch_pdl(time_sinusoid_kernel, dim3((n + 255) / 256), dim3(256), 0, st, out, batch, tv, dim); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 
@@ -500,7 +532,7 @@ cudaError_t gemv(const WT* W, const float* x, const float* bias, float* y, int N
   if (batch > 8) return cudaErrorInvalidValue;
   const size_t smem = (size_t)batch * K * sizeof(float);
   if (smem > 48 * 1024) return cudaErrorInvalidValue;
-  gemv_kernel<WT><<<(N + 7) / 8, 256, smem, st>>>(W, x, bias, y, N, K, batch, silu_in, silu_out);
+  { cudaError_t e_ = launch_pdl(gemv_kernel<WT>, dim3((N + 7) / 8), dim3(256), smem, st, W, x, bias, y, N, K, batch, silu_in, silu_out); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 template cudaError_t gemv<float>(const float*, const float*, const float*, float*, int, int, int, int, int,
@@ -511,7 +543,7 @@ template cudaError_t gemv<bf16>(const bf16*, const float*, const float*, float*,
 cudaError_t assemble_mods(const float* table, const float* e0, const float* htable, const float* e, float* mods,
                           float* hmods, int batch, int blocks, int D, cudaStream_t st) {
   const long n = (long)batch * blocks * 6 * D + (long)batch * 2 * D;
-  assemble_mods_kernel<<<grid_for(n, 256), 256, 0, st>>>(table, e0, htable, e, mods, hmods, batch, blocks, D);
+  { cudaError_t e_ = launch_pdl(assemble_mods_kernel, dim3(grid_for(n, 256)), dim3(256), 0, st, table, e0, htable, e, mods, hmods, batch, blocks, D); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 
@@ -520,7 +552,7 @@ cudaError_t prep_tokens(const float* x, const float* ref, const float* motion, i
                         int batch, int C, int L, int HW, cudaStream_t st) {
   if (C % 32 != 0) return cudaErrorInvalidValue;
   dim3 grid((L + 31) / 32, C / 32, batch);
-  prep_tokens_kernel<T><<<grid, dim3(32, 8), 0, st>>>(x, ref, motion, pin_frames, lat, tok, C, L, HW);
+  { cudaError_t e_ = launch_pdl(prep_tokens_kernel<T>, dim3(grid), dim3(dim3(32, 8)), 0, st, x, ref, motion, pin_frames, lat, tok, C, L, HW); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 template cudaError_t prep_tokens<float>(const float*, const float*, const float*, int, float*, float*, int, int, int,
@@ -532,7 +564,7 @@ template <typename T>
 cudaError_t euler_step(float* lat, const float* v, float dsig, int pinned_tokens, T* tok, int batch, int C, int L,
                        cudaStream_t st) {
   const long n = (long)batch * L * C;
-  euler_kernel<T><<<grid_for(n, 256), 256, 0, st>>>(lat, v, dsig, pinned_tokens, tok, C, L, n);
+  { cudaError_t e_ = launch_pdl(euler_kernel<T>, dim3(grid_for(n, 256)), dim3(256), 0, st, lat, v, dsig, pinned_tokens, tok, C, L, n); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 template cudaError_t euler_step<float>(float*, const float*, float, int, float*, int, int, int, cudaStream_t);
@@ -541,7 +573,7 @@ template cudaError_t euler_step<bf16>(float*, const float*, float, int, bf16*, i
 cudaError_t tokens_to_latent(const float* tok, float* out, int batch, int C, int L, cudaStream_t st) {
   if (C % 32 != 0) return cudaErrorInvalidValue;
   dim3 grid((L + 31) / 32, C / 32, batch);
-  tokens_to_latent_kernel<<<grid, dim3(32, 8), 0, st>>>(tok, out, C, L);
+  { cudaError_t e_ = launch_pdl(tokens_to_latent_kernel, dim3(grid), dim3(dim3(32, 8)), 0, st, tok, out, C, L); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 
@@ -550,8 +582,8 @@ cudaError_t gen_tensor(T* dst, long rows, long cols, long ld, uint64_t seed, int
                        bool round_bf16, cudaStream_t st) {
   const uint64_t base = seed ^ ((uint64_t)tid << 40);
   const long n = rows * cols;
-  gen_tensor_kernel<T><<<grid_for(n, 256), 256, 0, st>>>(dst, rows, cols, ld, base, kind, sqrt((double)fan),
-                                                         round_bf16);
+  { cudaError_t e_ = launch_pdl(gen_tensor_kernel<T>, dim3(grid_for(n, 256)), dim3(256), 0, st, dst, rows, cols, ld, base, kind, sqrt((double)fan),
+                                                         round_bf16); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 template cudaError_t gen_tensor<float>(float*, long, long, long, uint64_t, int, int, int, bool, cudaStream_t);
@@ -559,12 +591,12 @@ template cudaError_t gen_tensor<bf16>(bf16*, long, long, long, uint64_t, int, in
 
 cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st) {
   const int n = F * H * W * (pf + ph + pw);
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(tab, F, H, W, pf, ph, pw, (double)theta);
+  { cudaError_t e_ = launch_pdl(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, st, tab, F, H, W, pf, ph, pw, (double)theta); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 
 cudaError_t fill_f32(float* p, long n, float v, cudaStream_t st) {
-  fill_kernel<<<grid_for(n, 256), 256, 0, st>>>(p, n, v);
+  { cudaError_t e_ = launch_pdl(fill_kernel, dim3(grid_for(n, 256)), dim3(256), 0, st, p, n, v); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }
 
