@@ -486,6 +486,7 @@ int prepare_device(int dev) {
   if (dev < 32 && (done & (1u << dev))) return FH_OK;
   cudaError_t e = gemm_tc_prepare();
   if (e == cudaSuccess) e = attn_tc_prepare();
+  if (e == cudaSuccess) e = cross_attn_prepare();
   if (e != cudaSuccess) return fail(FH_ERR_CUDA, "kernel attribute setup: %s", cudaGetErrorString(e));
   if (dev < 32) done |= 1u << dev;
   return FH_OK;

@@ -10,13 +10,14 @@
 // attn_tc_kernel (bf16, sm_100a): one CTA per 128-query tile of one (stream, head).
 //   warp 0     TMA: the Q tile once, then K and V tiles (128 keys) double-buffered.
 //   warp 1     one thread issues tcgen05.mma: S_j = Q K_j^T into TMEM (double
-//              buffered), then O_j = P_j V_j into TMEM (double buffered; V is read
-//              MN-major straight from its [key][d] layout).
+//              buffered), then O_j = P_j V_j into TMEM (double buffered) with P_j
+//              read from TMEM as the A operand and V read MN-major straight from
+//              its [key][d] layout.
 //   warps 2-9  two threads per query row (one per warpgroup, 64 keys and 64 output
 //              dims each): S_j from TMEM, online softmax in base 2, P_j written as
-//              bf16 into 128-byte-swizzled shared memory for the next MMA, and O_j
-//              folded into a register accumulator that carries the running max
-//              correction.
+//              packed bf16 back into TMEM over the S_j columns it has consumed (so P
+//              is double-buffered with S at no cost), and O_j folded into a register
+//              accumulator that carries the running max correction.
 //   The MMA thread issues S_{j+1} before P_j V_j so the tensor core works while the
 //   softmax warps exponentiate.
 // attn_simt_kernel (fp32 or bf16 inputs, CUDA cores): one query row per thread, a
@@ -38,8 +39,7 @@ constexpr uint32_t TILE = 2 * PANEL;            // [128 rows x 128 bf16]
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + TILE;        // 2 buffers
 constexpr uint32_t OFF_V = OFF_K + 2 * TILE;    // 2 buffers
-constexpr uint32_t OFF_P = OFF_V + 2 * TILE;    // 1 buffer
-constexpr uint32_t OFF_RK = OFF_P + TILE;       // float rk[2][128]
+constexpr uint32_t OFF_RK = OFF_V + 2 * TILE;   // float rk[2][128]
 constexpr uint32_t OFF_MX = OFF_RK + 2 * 128 * 4;  // float [2][2][128] partial row maxima
 constexpr uint32_t OFF_LS = OFF_MX + 4 * 128 * 4;  // float [2][128] partial row sums
 constexpr uint32_t OFF_BAR = OFF_LS + 2 * 128 * 4;
@@ -72,11 +72,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint64_t* v_full = bars + 3;    // [2]
   uint64_t* kv_empty = bars + 5;  // [2]
   uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* s_free = bars + 9;    // [2]
   uint64_t* o_full = bars + 11;   // [2]
   uint64_t* o_free = bars + 13;   // [2]
   uint64_t* p_full = bars + 15;
-  uint64_t* p_free = bars + 16;
   uint64_t* rk_full = bars + 17;  // [2]
   uint64_t* rk_free = bars + 19;  // [2]
   uint64_t* mx_bar = bars + 21;   // [2]
@@ -98,12 +96,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mbar_init(&v_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], AT_SOFTMAX_THREADS);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], AT_SOFTMAX_THREADS);
     }
     mbar_init(p_full, AT_SOFTMAX_THREADS);
-    mbar_init(p_free, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&rk_full[i], AT_SOFTMAX_THREADS);
       mbar_init(&rk_free[i], AT_SOFTMAX_THREADS);
@@ -165,15 +161,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
       const uint32_t id_o = idesc_bf16_f32(128, 128, true);
       const uint32_t q_addr = smem_u32(smem + OFF_Q);
-      const uint32_t p_addr = smem_u32(smem + OFF_P);
       bool ok = mbar_wait(q_full, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       tc_fence_after();
       for (int j = 0; ok && j <= nkv; ++j) {
         if (j < nkv) {  // S_j = Q K_j^T
           const int bf = j & 1;
           const uint32_t par = (j >> 1) & 1;
+          // S_j overwrites the TMEM buffer that held S_{j-2} and P_{j-2}: K_j can only have been
+          // loaded into its buffer after P_{j-2} V_{j-2} completed (kv_empty), so it is free
           if (!mbar_wait(&k_full[bf], par, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
-          if (!mbar_wait(&s_free[bf], par ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(smem + OFF_K + bf * TILE);
 #pragma unroll
@@ -195,13 +191,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           const uint32_t v_addr = smem_u32(smem + OFF_V + bf * TILE);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t a_off = (kk >> 2) * PANEL + (kk & 3) * 32;  // 16 keys of P
+            // keys 16kk..16kk+15 of P_i: packed in columns 64*(kk/4) + 8*(kk%4) of S_i's buffer
+            const uint32_t a_tmem = tmem + bf * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
             const uint32_t b_off = kk * 16 * 128;                      // 16 key rows of V
-            tc_mma_f16(tmem + 256 + bf * 128, sdesc_kmajor_sw128(p_addr + a_off),
-                       sdesc_mnmajor_sw128(v_addr + b_off, PANEL), id_o, kk > 0 ? 1u : 0u);
+            tc_mma_f16_ts(tmem + 256 + bf * 128, a_tmem, sdesc_mnmajor_sw128(v_addr + b_off, PANEL), id_o,
+                          kk > 0 ? 1u : 0u);
           }
           tc_commit(&o_full[bf]);
-          tc_commit(p_free);
           tc_commit(&kv_empty[bf]);
         }
       }
@@ -221,8 +217,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     const float rq = row_rms(ssq, ssq_ld, (long)b * L + (qvalid ? qi : L - 1), 0, heads, inv_d, eps);
     const float qscale = rq * scale_log2;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint8_t* prow = smem + OFF_P + half * PANEL + (uint32_t)rl * 128;  // this half's 64 keys of P
-    const int sw = lane & 7;  // (row % 8) for the 128-byte swizzle; quarter*32 is a multiple of 8
     float* mxs = reinterpret_cast<float*>(smem + OFF_MX);  // [2 tiles][2 halves][128 rows]
     float* lss = reinterpret_cast<float*>(smem + OFF_LS);  // [2 halves][128 rows]
 
@@ -280,13 +274,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mx = fmaxf(mx, mxt[(1 - half) * 128 + rl]);
       const float m_new = fmaxf(m_run, mx * qscale);
       const float alpha = ex2(m_run - m_new);
-      // P_j overwrites the P buffer: wait until P_{j-1} V_{j-1} has consumed it
-      if (j >= 1) {
-        ok = mbar_wait(p_free, (j - 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-      }
-      // pass 2: probabilities, partial row sum, bf16 P into this half's swizzled panel
+      // pass 2: probabilities, partial row sum, packed bf16 P written over the consumed S columns
       float rs = 0.f;
 #pragma unroll 1
       for (int c = 0; c < 64; c += 32) {
@@ -299,19 +287,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           v[e] = p;
           rs += p;
         }
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = (c >> 3) + q;
-          __nv_bfloat162 hv[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) hv[u] = __floats2bfloat162_rn(v[q * 8 + 2 * u], v[q * 8 + 2 * u + 1]);
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ sw) << 4)) = *reinterpret_cast<uint4*>(hv);
+        for (int u = 0; u < 16; ++u) {
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
+          pk[u] = *reinterpret_cast<uint32_t*>(&h2);
         }
+        tmem_st16(s_t + (c >> 1), pk);  // columns already read by this half (c/2 < c + 32)
       }
       mbar_arrive(&rk_free[bf]);
+      tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&s_free[bf]);
-      fence_proxy_async_smem();
       mbar_arrive(p_full);
       l_run = l_run * alpha + rs;
       m_run = m_new;

@@ -55,6 +55,7 @@ cudaError_t attn_simt(const T* q, const T* k, const T* v, const float* ssq, int 
 // q [B*L, D] row-major with ssq_q [B*L, heads]; keys/values: rows (b*F + f)*A + a of
 // kv (row stride ldkv), key columns at koff, value columns at voff, with key partial
 // sums of squares ssq_k[row * ssq_k_ld + ssq_k_off + h]. out [B*L, D].
+cudaError_t cross_attn_prepare();  // shared-memory attribute, outside any stream capture
 template <typename T>
 cudaError_t cross_attn(const T* q, const float* ssq_q, const T* kv, long ldkv, int koff, int voff,
                        const float* ssq_k, int ssq_k_ld, int ssq_k_off, int batch, int heads, int L, int F, int A,

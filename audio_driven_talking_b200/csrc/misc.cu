@@ -87,109 +87,131 @@ __global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ ou
 // A token of latent frame f attends to frame f's A = 32 audio tokens only (gizai:flashhead,
 // opening paragraph: 5 latent frames of 32 audio tokens; reading R5). One CTA per (frame,
 // head, stream, chunk of XA_QPB queries) stages that frame's keys/values (fp32) and key RMS
-// factors in shared memory. One warp per query: lane a scores audio key a, the softmax is a
-// pair of warp reductions, and lane l accumulates output dims 4l..4l+3.
+// factors in shared memory. Each warp takes XA_QPW queries at once: for the scores lane a
+// owns audio key a and every float4 of k_a read from shared memory serves all XA_QPW
+// queries; for the output lane l owns dims 4l..4l+3 and every float4 of v_a serves all of
+// them, so shared-memory traffic per query is XA_QPW times smaller than one query at a time.
 constexpr int XA_WARPS = 8;
-constexpr int XA_QPW = 8;                    // queries per warp
+constexpr int XA_QPW = 8;                    // queries per warp, processed together
 constexpr int XA_QPB = XA_WARPS * XA_QPW;    // queries per CTA
+constexpr int XA_A = 32;                     // audio tokens per latent frame
+constexpr int XA_KS = 132;                   // padded row stride of staged keys (float4-aligned)
+constexpr size_t XA_SMEM = (size_t)XA_A * XA_KS * 4 + (size_t)XA_A * 128 * 4 + (size_t)XA_WARPS * XA_QPW * 128 * 4 +
+                           XA_A * 4;
+
+template <typename T>
+__device__ __forceinline__ float4 load4f(const T* p) {
+  if constexpr (sizeof(T) == 2) {
+    uint2 u = *reinterpret_cast<const uint2*>(p);
+    float2 a0 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+    float2 a1 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+    return make_float4(a0.x, a0.y, a1.x, a1.y);
+  } else {
+    return *reinterpret_cast<const float4*>(p);
+  }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(XA_WARPS * 32)
     cross_attn_kernel(const T* __restrict__ q, const float* __restrict__ ssq_q, const T* __restrict__ kv, long ldkv,
                       int koff, int voff, const float* __restrict__ ssq_k, int ssq_k_ld, int ssq_k_off, int heads,
                       int L, int F, int nqc, float eps, float scale, T* __restrict__ out) {
+  extern __shared__ __align__(16) float xa_smem[];
+  float* ks = xa_smem;                                   // [A][XA_KS]
+  float* vs = ks + XA_A * XA_KS;                         // [A][128]
+  float* qs = vs + XA_A * 128;                           // [warps][QPW][128]
+  float* rks = qs + XA_WARPS * XA_QPW * 128;             // [A]
   pdl_launch_dependents();
   pdl_wait();
-  constexpr int A = 32;
-  __shared__ float ks[A][129];
-  __shared__ __align__(16) float vs[A][128];
-  __shared__ float rks[A];
-  __shared__ float qs[XA_WARPS][128];
   const int f = blockIdx.x / nqc, qc = blockIdx.x % nqc;
   const int h = blockIdx.y, b = blockIdx.z;
   const int D = heads * 128;
   const float inv_d = 1.f / (float)D;
-  const long kv_row0 = ((long)b * F + f) * A;
+  const long kv_row0 = ((long)b * F + f) * XA_A;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int HW = L / F;
-  // issue every global load of this warp's queries up front (they are independent)
   const int n0 = qc * XA_QPB + warp * XA_QPW;
-  float4 qpre[XA_QPW];
-  float sqpre[XA_QPW];
+  // this warp's query slices and RMS partial sums, all loads in flight together
+  float4 qv[XA_QPW];
+  float sq[XA_QPW];
 #pragma unroll
   for (int i = 0; i < XA_QPW; ++i) {
     const int n = n0 + i < HW ? n0 + i : HW - 1;
     const long row = (long)b * L + (long)f * HW + n;
-    sqpre[i] = lane < heads ? ssq_q[row * heads + lane] : 0.f;
-    const T* qr = q + row * D + h * 128 + lane * 4;
-    if constexpr (sizeof(T) == 2) {
-      uint2 u = *reinterpret_cast<const uint2*>(qr);
-      float2 a0 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
-      float2 a1 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
-      qpre[i] = make_float4(a0.x, a0.y, a1.x, a1.y);
-    } else {
-      qpre[i] = *reinterpret_cast<const float4*>(qr);
-    }
+    sq[i] = lane < heads ? ssq_q[row * heads + lane] : 0.f;
+    qv[i] = load4f(q + row * D + h * 128 + lane * 4);
   }
-  for (int idx = threadIdx.x; idx < A * 16; idx += blockDim.x) {
-    const int a = idx >> 4, d = (idx & 15) * 8;
+  for (int idx = threadIdx.x; idx < XA_A * 32; idx += blockDim.x) {
+    const int a = idx >> 5, d = (idx & 31) * 4;
     const T* r = kv + (kv_row0 + a) * ldkv;
-    float tk[8], tv[8];
-    load8(r + koff + h * 128 + d, tk);
-    load8(r + voff + h * 128 + d, tv);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      ks[a][d + e] = tk[e];
-      vs[a][d + e] = tv[e];
-    }
+    *reinterpret_cast<float4*>(&ks[a * XA_KS + d]) = load4f(r + koff + h * 128 + d);
+    *reinterpret_cast<float4*>(&vs[a * 128 + d]) = load4f(r + voff + h * 128 + d);
   }
-  if (threadIdx.x < A) {
+  if (threadIdx.x < XA_A) {
     const float* p = ssq_k + (kv_row0 + threadIdx.x) * ssq_k_ld + ssq_k_off;
     float s = 0.f;
     for (int i = 0; i < heads; ++i) s += p[i];
     rks[threadIdx.x] = rsqrtf(s * inv_d + eps);
   }
+  float* qw = qs + warp * XA_QPW * 128;
+#pragma unroll
+  for (int i = 0; i < XA_QPW; ++i) *reinterpret_cast<float4*>(&qw[i * 128 + lane * 4]) = qv[i];
   __syncthreads();
+  if (n0 >= HW) return;
+
+  // scores: lane = audio key
+  float s[XA_QPW];
+#pragma unroll
+  for (int i = 0; i < XA_QPW; ++i) s[i] = 0.f;
+  const float* kr = ks + lane * XA_KS;
+#pragma unroll 4
+  for (int d = 0; d < 128; d += 4) {
+    const float4 k4 = *reinterpret_cast<const float4*>(kr + d);
+#pragma unroll
+    for (int i = 0; i < XA_QPW; ++i) {
+      const float4 q4 = *reinterpret_cast<const float4*>(qw + i * 128 + d);
+      s[i] = fmaf(q4.x, k4.x, fmaf(q4.y, k4.y, fmaf(q4.z, k4.z, fmaf(q4.w, k4.w, s[i]))));
+    }
+  }
   const float rk = rks[lane] * scale;
+#pragma unroll
+  for (int i = 0; i < XA_QPW; ++i) {
+    const float rq = rsqrtf(warp_sum(sq[i]) * inv_d + eps);
+    const float si = s[i] * rq * rk;
+    const float m = warp_max(si);
+    const float p = expf(si - m);
+    s[i] = p / warp_sum(p);  // normalised weight of key `lane` for query i
+  }
+  // output: lane = 4 dims
+  float4 o[XA_QPW];
+#pragma unroll
+  for (int i = 0; i < XA_QPW; ++i) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int a = 0; a < XA_A; ++a) {
+    const float4 vv = *reinterpret_cast<const float4*>(&vs[a * 128 + lane * 4]);
+#pragma unroll
+    for (int i = 0; i < XA_QPW; ++i) {
+      const float pa = __shfl_sync(0xffffffffu, s[i], a);
+      o[i].x = fmaf(pa, vv.x, o[i].x);
+      o[i].y = fmaf(pa, vv.y, o[i].y);
+      o[i].z = fmaf(pa, vv.z, o[i].z);
+      o[i].w = fmaf(pa, vv.w, o[i].w);
+    }
+  }
 #pragma unroll
   for (int i = 0; i < XA_QPW; ++i) {
     const int n = n0 + i;
     if (n >= HW) break;
-    const long row = (long)b * L + (long)f * HW + n;
-    const float rq = rsqrtf(warp_sum(sqpre[i]) * inv_d + eps);
-    const float4 qv = qpre[i];
-    __syncwarp();
-    *reinterpret_cast<float4*>(&qs[warp][lane * 4]) = qv;
-    __syncwarp();
-    // lane = audio key
-    float s = 0.f;
-#pragma unroll 16
-    for (int d = 0; d < 128; ++d) s = fmaf(qs[warp][d], ks[lane][d], s);
-    s *= rq * rk;
-    const float m = warp_max(s);
-    const float p = expf(s - m);
-    const float inv_z = 1.f / warp_sum(p);
-    // lane = 4 output dims
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-    for (int a = 0; a < A; ++a) {
-      const float pa = __shfl_sync(0xffffffffu, p, a);
-      const float4 vv = *reinterpret_cast<const float4*>(&vs[a][lane * 4]);
-      o.x = fmaf(pa, vv.x, o.x);
-      o.y = fmaf(pa, vv.y, o.y);
-      o.z = fmaf(pa, vv.z, o.z);
-      o.w = fmaf(pa, vv.w, o.w);
-    }
-    T* dst = out + row * D + h * 128 + lane * 4;
+    T* dst = out + ((long)b * L + (long)f * HW + n) * D + h * 128 + lane * 4;
     if constexpr (sizeof(T) == 2) {
-      __nv_bfloat162 h0 = __floats2bfloat162_rn(o.x * inv_z, o.y * inv_z);
-      __nv_bfloat162 h1 = __floats2bfloat162_rn(o.z * inv_z, o.w * inv_z);
+      __nv_bfloat162 h0 = __floats2bfloat162_rn(o[i].x, o[i].y);
+      __nv_bfloat162 h1 = __floats2bfloat162_rn(o[i].z, o[i].w);
       uint2 u;
       u.x = *reinterpret_cast<uint32_t*>(&h0);
       u.y = *reinterpret_cast<uint32_t*>(&h1);
       *reinterpret_cast<uint2*>(dst) = u;
     } else {
-      *reinterpret_cast<float4*>(dst) = make_float4(o.x * inv_z, o.y * inv_z, o.z * inv_z, o.w * inv_z);
+      *reinterpret_cast<float4*>(dst) = o[i];
     }
   }
 }
@@ -479,18 +501,25 @@ cudaError_t gemm_simt(const float* A, long lda, const float* W, long ldw, int M,
   return cudaGetLastError();
 }
 
+cudaError_t cross_attn_prepare() {
+  cudaError_t e = cudaFuncSetAttribute(cross_attn_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)XA_SMEM);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(cross_attn_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)XA_SMEM);
+}
+
 template <typename T>
 cudaError_t cross_attn(const T* q, const float* ssq_q, const T* kv, long ldkv, int koff, int voff,
                        const float* ssq_k, int ssq_k_ld, int ssq_k_off, int batch, int heads, int L, int F, int A,
                        float eps, T* out, cudaStream_t st) {
-  if (A != 32 || heads > 32) return cudaErrorInvalidValue;
+  if (A != XA_A || heads > 32) return cudaErrorInvalidValue;
   const int HW = L / F;
   const int nqc = (HW + XA_QPB - 1) / XA_QPB;
   dim3 grid(F * nqc, heads, batch);
-  { cudaError_t e_ = launch_pdl(cross_attn_kernel<T>, dim3(grid), dim3(XA_WARPS * 32), 0, st, q, ssq_q, kv, ldkv, koff, voff, ssq_k, ssq_k_ld, ssq_k_off,
-                                                      heads, L, F, nqc, eps, 1.f / sqrtf(128.f), out); if (e_ != cudaSuccess) return e_; }
-  return cudaGetLastError();
+  return launch_pdl(cross_attn_kernel<T>, grid, dim3(XA_WARPS * 32), XA_SMEM, st, q, ssq_q, kv, ldkv, koff, voff,
+                    ssq_k, ssq_k_ld, ssq_k_off, heads, L, F, nqc, eps, 1.f / sqrtf(128.f), out);
 }
+
 template cudaError_t cross_attn<float>(const float*, const float*, const float*, long, int, int, const float*, int,
                                        int, int, int, int, int, int, float, float*, cudaStream_t);
 template cudaError_t cross_attn<bf16>(const bf16*, const float*, const bf16*, long, int, int, const float*, int,
