@@ -336,7 +336,12 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
   const float eps = m->cfg.eps;
 
   // self-attention branch
-  LAUNCH(norm_rows<T>(x, h, M, D, L, 0, mods + 0 * D, mods + 1 * D, mbs, nullptr, nullptr, eps, st));
+  {
+    const int ti = timed_begin(m, 6, st);
+    cudaError_t e = norm_rows<T>(x, h, M, D, L, 0, mods + 0 * D, mods + 1 * D, mbs, nullptr, nullptr, eps, st);
+    timed_end(m, ti, st);
+    LAUNCH(e);
+  }
   {
     EpiParams ep = epi0(L);
     ep.bias = bw.bqkv;
@@ -383,11 +388,16 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
     ep.ssq_ld = NH;
     ep.norm_period = D;
     ep.norm_count = D;
-    RUN(run_gemm(m, &P.m_h, h, D, &bw.m_cq, bw.wcq, D, M, D, D, EPI_NORM, m->bf16, ep, st, 0));
+    RUN(run_gemm(m, &P.m_h, h, D, &bw.m_cq, bw.wcq, D, M, D, D, EPI_NORM, m->bf16, ep, st, 7));
   }
-  LAUNCH(cross_attn<T>(at<T>(ws, w.cq), at<float>(ws, w.ssq_cq), at<T>(ws, w.ckv), (long)m->NB * 2 * D, k * 2 * D,
-                       k * 2 * D + D, at<float>(ws, w.ssq_ckv), m->NB * 2 * NH, k * 2 * NH, B, NH, L, m->F, m->A,
-                       eps, attn, st));
+  {
+    const int ti = timed_begin(m, 5, st);
+    cudaError_t e = cross_attn<T>(at<T>(ws, w.cq), at<float>(ws, w.ssq_cq), at<T>(ws, w.ckv), (long)m->NB * 2 * D,
+                                  k * 2 * D, k * 2 * D + D, at<float>(ws, w.ssq_ckv), m->NB * 2 * NH, k * 2 * NH, B,
+                                  NH, L, m->F, m->A, eps, attn, st);
+    timed_end(m, ti, st);
+    LAUNCH(e);
+  }
   {
     EpiParams ep = epi0(L);
     ep.bias = bw.bco;
@@ -510,7 +520,7 @@ int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** ou
       c.dim / 128 > 16 || c.dim > 1536 * 4)
     return fail(FH_ERR_SHAPE, "configuration outside the supported set");
   const int L = c.frames * c.lat_h * c.lat_w;
-  if (L > 16384) return fail(FH_ERR_SHAPE, "token count %d above 16384", L);
+  if (L > 8192) return fail(FH_ERR_SHAPE, "token count %d above 8192", L);
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || c.device < 0 || c.device >= ndev)
     return fail(FH_ERR_UNSUPPORTED, "no CUDA device %d", c.device);
@@ -944,7 +954,7 @@ int fh_dit_sync(fh_dit* m, void* stream) {
 int fh_dit_last_launch_count(const fh_dit* m) { return m ? m->last_launches : 0; }
 
 int fh_dit_set_timing(fh_dit* m, int kernel_class) {
-  if (!m || kernel_class < 0 || kernel_class > 4) return fail(FH_ERR_ARG, "bad timing class");
+  if (!m || kernel_class < 0 || kernel_class > 7) return fail(FH_ERR_ARG, "bad timing class");
   cudaSetDevice(m->device);
   if (kernel_class && m->events.empty()) {
     m->events.resize(2048);

@@ -39,11 +39,12 @@ constexpr uint32_t TILE = 2 * PANEL;            // [128 rows x 128 bf16]
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + TILE;        // 2 buffers
 constexpr uint32_t OFF_V = OFF_K + 2 * TILE;    // 2 buffers
-constexpr uint32_t OFF_RK = OFF_V + 2 * TILE;   // float rk[2][128]
-constexpr uint32_t OFF_MX = OFF_RK + 2 * 128 * 4;  // float [2][2][128] partial row maxima
+constexpr uint32_t OFF_MX = OFF_V + 2 * TILE;   // float [2][2][128] partial row maxima
 constexpr uint32_t OFF_LS = OFF_MX + 4 * 128 * 4;  // float [2][128] partial row sums
 constexpr uint32_t OFF_BAR = OFF_LS + 2 * 128 * 4;
-constexpr uint32_t AT_SMEM = OFF_BAR + 256 + 1024;
+constexpr uint32_t OFF_RKALL = OFF_BAR + 256;   // float rk[round_up(L, 128)]: every key's RMS factor
+constexpr int AT_MAX_L = 8192;
+constexpr uint32_t AT_SMEM = OFF_RKALL + AT_MAX_L * 4 + 1024;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -65,18 +66,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                    int L, float eps, float scale_log2, bf16* __restrict__ out, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* rk_s = reinterpret_cast<float*>(smem + OFF_RK);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* k_empty = bars + 5;   // [2] K buffer free (S MMA done)
+  uint64_t* v_empty = bars + 9;   // [2] V buffer free (P.V MMA done); also orders S-buffer reuse
   uint64_t* s_full = bars + 7;    // [2]
   uint64_t* o_full = bars + 11;   // [2]
   uint64_t* o_free = bars + 13;   // [2]
   uint64_t* p_full = bars + 15;
-  uint64_t* rk_full = bars + 17;  // [2]
-  uint64_t* rk_free = bars + 19;  // [2]
+  uint64_t* rk_full = bars + 17;  // every key's RMS factor staged
   uint64_t* mx_bar = bars + 21;   // [2]
   uint64_t* l_bar = bars + 23;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
@@ -94,18 +94,18 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&o_full[i], 1);
       mbar_init(&o_free[i], AT_SOFTMAX_THREADS);
     }
     mbar_init(p_full, AT_SOFTMAX_THREADS);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&rk_full[i], AT_SOFTMAX_THREADS);
-      mbar_init(&rk_free[i], AT_SOFTMAX_THREADS);
       mbar_init(&mx_bar[i], AT_SOFTMAX_THREADS);
     }
     mbar_init(l_bar, AT_SOFTMAX_THREADS);
+    mbar_init(rk_full, AT_SOFTMAX_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -125,33 +125,49 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
+      int kiss = 0, viss = 0;  // K and V tiles issued
       mbar_expect_tx(q_full, TILE);
       tma_load_2d(&tmQ, q_full, smem + OFF_Q, 0, bh_row0 + qt * AT_BQ);
       tma_load_2d(&tmQ, q_full, smem + OFF_Q + PANEL, 64, bh_row0 + qt * AT_BQ);
-      for (int j = 0; j < nkv; ++j) {
+      // order K_0, K_1, V_0, K_2, V_1, ...: the MMA issues S_{j+1} before P_j V_j
+      auto load_k = [&](int j) -> bool {
         const int bf = j & 1;
-        if (!mbar_wait(&kv_empty[bf], ((j >> 1) & 1) ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
+        if (!mbar_wait(&k_empty[bf], ((j >> 1) & 1) ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) return false;
         const int r0 = bh_row0 + j * AT_BK;
         mbar_expect_tx(&k_full[bf], TILE);
         tma_load_2d(&tmK, &k_full[bf], smem + OFF_K + bf * TILE, 0, r0);
         tma_load_2d(&tmK, &k_full[bf], smem + OFF_K + bf * TILE + PANEL, 64, r0);
+        kiss = j + 1;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int bf = j & 1;
+        if (!mbar_wait(&v_empty[bf], ((j >> 1) & 1) ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) return false;
+        const int r0 = bh_row0 + j * AT_BK;
         mbar_expect_tx(&v_full[bf], TILE);
         tma_load_2d(&tmV, &v_full[bf], smem + OFF_V + bf * TILE, 0, r0);
         tma_load_2d(&tmV, &v_full[bf], smem + OFF_V + bf * TILE + PANEL, 64, r0);
-        issued = j + 1;
+        viss = j + 1;
+        return true;
+      };
+      if (load_k(0)) {
+        for (int j = 0; j < nkv; ++j) {
+          if (j + 1 < nkv && !load_k(j + 1)) break;
+          if (!load_v(j)) break;
+        }
       }
       if (*abort_flag) {
         uint64_t t0 = globaltimer();
         while (!mbar_try_wait(q_full, 0) && globaltimer() - t0 < FH_WAIT_LIMIT_NS) {
         }
-        for (int j = issued - 2 < 0 ? 0 : issued - 2; j < issued; ++j) {
-          const uint32_t par = (j >> 1) & 1;
+        for (int j = kiss - 2 < 0 ? 0 : kiss - 2; j < kiss; ++j) {
           t0 = globaltimer();
-          while (!mbar_try_wait(&k_full[j & 1], par) && globaltimer() - t0 < FH_WAIT_LIMIT_NS) {
+          while (!mbar_try_wait(&k_full[j & 1], (j >> 1) & 1) && globaltimer() - t0 < FH_WAIT_LIMIT_NS) {
           }
+        }
+        for (int j = viss - 2 < 0 ? 0 : viss - 2; j < viss; ++j) {
           t0 = globaltimer();
-          while (!mbar_try_wait(&v_full[j & 1], par) && globaltimer() - t0 < FH_WAIT_LIMIT_NS) {
+          while (!mbar_try_wait(&v_full[j & 1], (j >> 1) & 1) && globaltimer() - t0 < FH_WAIT_LIMIT_NS) {
           }
         }
       }
@@ -167,9 +183,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         if (j < nkv) {  // S_j = Q K_j^T
           const int bf = j & 1;
           const uint32_t par = (j >> 1) & 1;
-          // S_j overwrites the TMEM buffer that held S_{j-2} and P_{j-2}: K_j can only have been
-          // loaded into its buffer after P_{j-2} V_{j-2} completed (kv_empty), so it is free
           if (!mbar_wait(&k_full[bf], par, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
+          // S_j overwrites the TMEM buffer that held S_{j-2} and P_{j-2}: wait for P_{j-2} V_{j-2}
+          if (j >= 2 && !mbar_wait(&v_empty[bf], par ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
           tc_fence_after();
           const uint32_t k_addr = smem_u32(smem + OFF_K + bf * TILE);
 #pragma unroll
@@ -179,6 +195,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                        kk > 0 ? 1u : 0u);
           }
           tc_commit(&s_full[bf]);
+          tc_commit(&k_empty[bf]);
         }
         if (j >= 1) {  // O_i = P_i V_i for i = j - 1
           const int i = j - 1;
@@ -198,7 +215,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
                           kk > 0 ? 1u : 0u);
           }
           tc_commit(&o_full[bf]);
-          tc_commit(&kv_empty[bf]);
+          tc_commit(&v_empty[bf]);
         }
       }
     }
@@ -220,8 +237,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     float* mxs = reinterpret_cast<float*>(smem + OFF_MX);  // [2 tiles][2 halves][128 rows]
     float* lss = reinterpret_cast<float*>(smem + OFF_LS);  // [2 halves][128 rows]
 
-    // per-key RMS factors of the K tiles, staged one tile ahead through two buffers
-    if (t < AT_BK) rk_s[t] = t < L ? row_rms(ssq, ssq_ld, (long)b * L + t, heads, heads, inv_d, eps) : 0.f;
+    // every key's RMS factor, once per CTA (the keys are shared by all tiles of the row)
+    float* rk_all = reinterpret_cast<float*>(smem + OFF_RKALL);
+    for (int key = t; key < nkv * AT_BK; key += AT_SOFTMAX_THREADS)
+      rk_all[key] = key < L ? row_rms(ssq, ssq_ld, (long)b * L + key, heads, heads, inv_d, eps) : 0.f;
     mbar_arrive(&rk_full[0]);
     float o[64];
 #pragma unroll
@@ -229,23 +248,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
 
-    for (int j = 0; j < nkv; ++j) {
-      if (j + 1 < nkv) {
-        const int nb = (j + 1) & 1;
-        if (j >= 1) {  // tile j-1 used this buffer
-          ok = mbar_wait(&rk_free[nb], ((j - 1) >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-        }
-        const int key = (j + 1) * AT_BK + t;
-        if (t < AT_BK)
-          rk_s[nb * 128 + t] = key < L ? row_rms(ssq, ssq_ld, (long)b * L + key, heads, heads, inv_d, eps) : 0.f;
-        mbar_arrive(&rk_full[nb]);
-      }
-      ok = mbar_wait(&rk_full[j & 1], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      const float* rk = rk_s + (j & 1) * 128 + half * 64;
+    ok = mbar_wait(&rk_full[0], 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+    ok = __all_sync(0xffffffffu, ok);
+    for (int j = 0; ok && j < nkv; ++j) {
+      const float* rk = rk_all + j * AT_BK + half * 64;
       const int bf = j & 1;
       const uint32_t par = (j >> 1) & 1;
       ok = mbar_wait(&s_full[bf], par, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
@@ -254,16 +260,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       tc_fence_after();
       const uint32_t s_t = tmem + lane_off + bf * 128 + half * 64;
       const int kvalid = L - j * AT_BK - half * 64;  // keys of this half-tile that exist
-      // pass 1: partial row max over this half's keys, then exchange with the other half
+      // this half's 64 scores of the row, one batched TMEM read kept in registers for both passes
+      float sa[32], sb[32];
+      tmem_ld32(s_t, sa);
+      tmem_ld32(s_t + 32, sb);
+      tc_wait_ld();
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 64; c += 32) {
-        float v[32];
-        tmem_ld32(s_t + c, v);
-        tc_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (c + e < kvalid) mx = fmaxf(mx, v[e] * rk[c + e]);
+      for (int e = 0; e < 32; ++e) {
+        if (e < kvalid) mx = fmaxf(mx, sa[e] * rk[e]);
+        if (e + 32 < kvalid) mx = fmaxf(mx, sb[e] * rk[e + 32]);
       }
       float* mxt = mxs + (j & 1) * 256;
       mxt[half * 128 + rl] = mx;
@@ -274,28 +280,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mx = fmaxf(mx, mxt[(1 - half) * 128 + rl]);
       const float m_new = fmaxf(m_run, mx * qscale);
       const float alpha = ex2(m_run - m_new);
-      // pass 2: probabilities, partial row sum, packed bf16 P written over the consumed S columns
+      // probabilities, partial row sum, packed bf16 P written over the consumed S columns
       float rs = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 64; c += 32) {
-        float v[32];
-        tmem_ld32(s_t + c, v);
-        tc_wait_ld();
+      uint32_t pa[16], pb2[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p = (c + e < kvalid) ? ex2(v[e] * rk[c + e] * qscale - m_new) : 0.f;
-          v[e] = p;
-          rs += p;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * u], v[2 * u + 1]);
-          pk[u] = *reinterpret_cast<uint32_t*>(&h2);
-        }
-        tmem_st16(s_t + (c >> 1), pk);  // columns already read by this half (c/2 < c + 32)
+      for (int u = 0; u < 16; ++u) {
+        const int e0 = 2 * u, e1 = 2 * u + 1;
+        const float p0 = e0 < kvalid ? ex2(sa[e0] * rk[e0] * qscale - m_new) : 0.f;
+        const float p1 = e1 < kvalid ? ex2(sa[e1] * rk[e1] * qscale - m_new) : 0.f;
+        const float q0 = e0 + 32 < kvalid ? ex2(sb[e0] * rk[e0 + 32] * qscale - m_new) : 0.f;
+        const float q1 = e1 + 32 < kvalid ? ex2(sb[e1] * rk[e1 + 32] * qscale - m_new) : 0.f;
+        rs += (p0 + p1) + (q0 + q1);
+        __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
+        __nv_bfloat162 h1 = __floats2bfloat162_rn(q0, q1);
+        pa[u] = *reinterpret_cast<uint32_t*>(&h0);
+        pb2[u] = *reinterpret_cast<uint32_t*>(&h1);
       }
-      mbar_arrive(&rk_free[bf]);
+      tmem_st16(s_t, pa);        // keys 0..31 of this half -> columns 0..15 (already read)
+      tmem_st16(s_t + 16, pb2);  // keys 32..63 -> columns 16..31
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -309,13 +311,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const uint32_t o_t = tmem + lane_off + 256 + pb * 128 + half * 64;
-#pragma unroll
-        for (int c = 0; c < 64; c += 32) {
-          float v[32];
-          tmem_ld32(o_t + c, v);
+        {
+          float oa[32], ob[32];
+          tmem_ld32(o_t, oa);
+          tmem_ld32(o_t + 32, ob);
           tc_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[c + e] = (o[c + e] + v[e]) * alpha;
+          for (int e = 0; e < 32; ++e) {
+            o[e] = (o[e] + oa[e]) * alpha;
+            o[e + 32] = (o[e + 32] + ob[e]) * alpha;
+          }
         }
         tc_fence_before();
         mbar_arrive(&o_free[pb]);
@@ -449,6 +454,7 @@ cudaError_t attn_tc_prepare() {
 cudaError_t attn_tc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const float* ssq,
                     int ssq_ld, int batch, int heads, int L, float eps, bf16* out, unsigned* err,
                     cudaStream_t st) {
+  if (L > AT_MAX_L) return cudaErrorInvalidValue;
   const float scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   dim3 grid((L + AT_BQ - 1) / AT_BQ, heads, batch);
   { cudaError_t e_ = launch_pdl(attn_tc_kernel, dim3(grid), dim3(AT_THREADS), AT_SMEM, st, q, k, v, ssq, ssq_ld, heads, L, eps, scale_log2, out, err); if (e_ != cudaSuccess) return e_; }

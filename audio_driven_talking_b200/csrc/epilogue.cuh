@@ -124,6 +124,27 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0,
   }
 }
 
+// EPI_RESID with the row's residual already in registers (xr: 8 float4 = these 32 columns):
+// x += gate * (acc + bias), stored back.
+__device__ __forceinline__ void epi_resid_chunk_pref(const EpiParams& p, int row, int col0, float (&v)[32],
+                                                     float4* xr) {
+  const float* b = p.bias + col0;
+  float* r = p.resid + (long)row * p.ldr + col0;
+  const float* g = p.gate ? p.gate + (long)(row / p.rows_per_batch) * p.gate_bstride + col0 : nullptr;
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float4 bb = *reinterpret_cast<const float4*>(b + j);
+    float4 a = make_float4(v[j] + bb.x, v[j + 1] + bb.y, v[j + 2] + bb.z, v[j + 3] + bb.w);
+    if (g) {
+      const float4 gg = *reinterpret_cast<const float4*>(g + j);
+      a.x *= gg.x; a.y *= gg.y; a.z *= gg.z; a.w *= gg.w;
+    }
+    float4 x = xr[j >> 2];
+    x.x += a.x; x.y += a.y; x.z += a.z; x.w += a.w;
+    *reinterpret_cast<float4*>(r + j) = x;
+  }
+}
+
 template <int KIND>
 __device__ __forceinline__ void epi_group_end(const EpiParams& p, int row, int gcol0, float ssq_acc) {
   if constexpr (KIND == EPI_NORM || KIND == EPI_QKV) {

@@ -191,24 +191,42 @@ __global__ void __launch_bounds__(192, 1)
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
-      bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
-      if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld below is warp-collective
-      tc_fence_after();
       const int m0 = (tile % num_m) * BM;
       const int n0 = (tile / num_m) * BN;
       const int row = m0 + quarter * 32 + lane;
       const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-#pragma unroll 1
-      for (int g = 0; g < BN; g += 128) {
-        float ssq = 0.f;
-#pragma unroll 1
+      if constexpr (KIND == EPI_RESID && BN == 128) {
+        // the residual row segment does not depend on the MMAs: fetch it while they run
+        float4 xr[32];
+        const float4* xrow = reinterpret_cast<const float4*>(ep.resid + (long)(row < M ? row : 0) * ep.ldr + n0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) xr[i] = xrow[i];
+        bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+        if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld below is warp-collective
+        tc_fence_after();
+#pragma unroll
         for (int c = 0; c < 128; c += 32) {
           float v[32];
-          tmem_ld32(tb + g + c, v);
+          tmem_ld32(tb + c, v);
           tc_wait_ld();
-          if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
+          if (row < M) epi_resid_chunk_pref(ep, row, n0 + c, v, &xr[c >> 2]);
         }
-        if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
+      } else {
+        bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+        if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld below is warp-collective
+        tc_fence_after();
+#pragma unroll 1
+        for (int g = 0; g < BN; g += 128) {
+          float ssq = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            float v[32];
+            tmem_ld32(tb + g + c, v);
+            tc_wait_ld();
+            if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
+          }
+          if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

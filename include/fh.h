@@ -166,7 +166,8 @@ int fh_dit_last_launch_count(const fh_dit* m);
 
 /* Optional per-launch timing of one kernel class inside fh_sample_slice, for
  * roofline reporting: 0 off, 1 the gated-residual GEMMs (O-proj, cross-O, FFN2),
- * 2 the FFN1 GEMM, 3 the QKV GEMM, 4 self-attention. Changing it re-records
+ * 2 the FFN1 GEMM, 3 the QKV GEMM, 4 self-attention, 5 cross-attention, 6 the
+ * first row norm of each block, 7 the cross-Q GEMM. Changing it re-records
  * graphs. fh_dit_get_timing returns the mean device time (microseconds) and count
  * of that class's launches in the last completed fh_sample_slice call. */
 int fh_dit_set_timing(fh_dit* m, int kernel_class);
