@@ -106,6 +106,7 @@ def load_library() -> ctypes.CDLL:
         "fh_last_error": (ctypes.c_char_p, []),
         "fh_op_linear": (I, [P, P, P, P, I, I, I, I, P]),
         "fh_dit_block_forward_noalloc": (I, [P, I, P, P, P, P, I, P]),
+        "fh_dit_probe_wait_timeout": (I, [P, P]),
         "fh_op_attention": (I, [P, P, P, P, P, I, I, I, F, I, P]),
     }
     for name, (res, args) in sig.items():
@@ -226,6 +227,10 @@ class DiT:
 
     def sync(self, stream=None):
         _check(load_library().fh_dit_sync(self._h, _stream(stream)))
+
+    def probe_wait_timeout(self, stream=None):
+        """Make one bounded kernel wait run out (test of the failure-detection path)."""
+        _check(load_library().fh_dit_probe_wait_timeout(self._h, _stream(stream)))
 
     @property
     def last_launch_count(self) -> int:

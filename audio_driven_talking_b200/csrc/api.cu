@@ -981,6 +981,13 @@ int fh_dit_get_timing(fh_dit* m, double* mean_us, int* launches) {
   return FH_OK;
 }
 
+int fh_dit_probe_wait_timeout(fh_dit* m, void* stream) {
+  if (!m) return fail(FH_ERR_ARG, "null model");
+  if (cudaSetDevice(m->device) != cudaSuccess) return fail(FH_ERR_CUDA, "cudaSetDevice failed");
+  CK(wait_probe(m->err_dev, reinterpret_cast<cudaStream_t>(stream)));
+  return FH_OK;
+}
+
 // ------------------------------------------------------------ operator entry points
 int fh_op_linear(const void* A, const void* W, const float* bias, float* out, int M, int N, int K, int dtype,
                  void* stream) {

@@ -265,12 +265,27 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       tmem_ld32(s_t, sa);
       tmem_ld32(s_t + 32, sb);
       tc_wait_ld();
-      float mx = -INFINITY;
+      // scaled scores r_k * (q.k); keys past the end of the sequence get -inf (only the last tile)
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        if (e < kvalid) mx = fmaxf(mx, sa[e] * rk[e]);
-        if (e + 32 < kvalid) mx = fmaxf(mx, sb[e] * rk[e + 32]);
+        sa[e] *= rk[e];
+        sb[e] *= rk[e + 32];
       }
+      if (kvalid < 64) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if (e >= kvalid) sa[e] = -INFINITY;
+          if (e + 32 >= kvalid) sb[e] = -INFINITY;
+        }
+      }
+      // row max as a tree (independent chains)
+      float m8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        m8[u] = fmaxf(fmaxf(sa[u], sa[u + 8]), fmaxf(sa[u + 16], sa[u + 24]));
+        m8[u] = fmaxf(m8[u], fmaxf(fmaxf(sb[u], sb[u + 8]), fmaxf(sb[u + 16], sb[u + 24])));
+      }
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       float* mxt = mxs + (j & 1) * 256;
       mxt[half * 128 + rl] = mx;
       mbar_arrive(&mx_bar[j & 1]);
@@ -280,22 +295,23 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mx = fmaxf(mx, mxt[(1 - half) * 128 + rl]);
       const float m_new = fmaxf(m_run, mx * qscale);
       const float alpha = ex2(m_run - m_new);
-      // probabilities, partial row sum, packed bf16 P written over the consumed S columns
-      float rs = 0.f;
+      // probabilities (ex2 of -inf is 0), four independent partial sums, packed bf16 P
+      // written over the consumed S columns
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pa[16], pb2[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        const int e0 = 2 * u, e1 = 2 * u + 1;
-        const float p0 = e0 < kvalid ? ex2(sa[e0] * rk[e0] * qscale - m_new) : 0.f;
-        const float p1 = e1 < kvalid ? ex2(sa[e1] * rk[e1] * qscale - m_new) : 0.f;
-        const float q0 = e0 + 32 < kvalid ? ex2(sb[e0] * rk[e0 + 32] * qscale - m_new) : 0.f;
-        const float q1 = e1 + 32 < kvalid ? ex2(sb[e1] * rk[e1 + 32] * qscale - m_new) : 0.f;
-        rs += (p0 + p1) + (q0 + q1);
+        const float p0 = ex2(fmaf(sa[2 * u], qscale, -m_new));
+        const float p1 = ex2(fmaf(sa[2 * u + 1], qscale, -m_new));
+        const float q0 = ex2(fmaf(sb[2 * u], qscale, -m_new));
+        const float q1 = ex2(fmaf(sb[2 * u + 1], qscale, -m_new));
+        rs4[u & 3] += (p0 + p1) + (q0 + q1);
         __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
         __nv_bfloat162 h1 = __floats2bfloat162_rn(q0, q1);
         pa[u] = *reinterpret_cast<uint32_t*>(&h0);
         pb2[u] = *reinterpret_cast<uint32_t*>(&h1);
       }
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tmem_st16(s_t, pa);        // keys 0..31 of this half -> columns 0..15 (already read)
       tmem_st16(s_t + 16, pb2);  // keys 32..63 -> columns 16..31
       tc_wait_st();

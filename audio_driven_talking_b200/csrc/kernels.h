@@ -98,5 +98,6 @@ cudaError_t gen_tensor(T* dst, long rows, long cols, long ld, uint64_t seed, int
                        bool round_bf16, cudaStream_t st);
 cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st);
 cudaError_t fill_f32(float* p, long n, float v, cudaStream_t st);
+cudaError_t wait_probe(unsigned* err, cudaStream_t st);
 
 }  // namespace fh

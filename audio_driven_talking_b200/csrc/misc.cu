@@ -477,6 +477,20 @@ __global__ void __launch_bounds__(128) gemm_simt_kernel(const float* __restrict_
   if (q == 0 && row < M) epi_group_end<KIND>(ep, row, n0, ssq_s[0][r] + ssq_s[1][r] + ssq_s[2][r] + ssq_s[3][r]);
 }
 
+// One CTA waits on an mbarrier that nothing arrives at: the bounded wait of the
+// production kernels runs out, latches its error bit and the kernel returns normally.
+__global__ void wait_probe_kernel(unsigned* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+}
+
 inline int grid_for(long n, int block) {
   long g = (n + block - 1) / block;
   if (g > 148 * 16) g = 148 * 16;
@@ -621,6 +635,11 @@ template cudaError_t gen_tensor<bf16>(bf16*, long, long, long, uint64_t, int, in
 cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st) {
   const int n = F * H * W * (pf + ph + pw);
   { cudaError_t e_ = launch_pdl(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, st, tab, F, H, W, pf, ph, pw, (double)theta); if (e_ != cudaSuccess) return e_; }
+  return cudaGetLastError();
+}
+
+cudaError_t wait_probe(unsigned* err, cudaStream_t st) {
+  wait_probe_kernel<<<1, 32, 0, st>>>(err);
   return cudaGetLastError();
 }
 

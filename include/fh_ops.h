@@ -32,6 +32,15 @@ int fh_op_linear(const void* A, const void* W, const float* bias, float* out, in
 int fh_op_attention(const void* q, const void* k, const void* v, const float* ssq, void* out, int batch,
                     int heads, int L, float eps, int dtype, void* stream);
 
+/* Failure-detection check (no counterpart on the pages; reading of the pages'
+ * reject-don't-hang stance): launches one CTA whose mbarrier wait has no arriving
+ * party. The kernel's bounded wait (the same one every production kernel uses, about
+ * one second of %globaltimer) runs out, latches the timeout bit into the model's
+ * device-visible error word and the kernel returns; nothing faults or hangs. The next
+ * fh_dit_sync on `stream` reports FH_ERR_TIMEOUT once and clears the word. */
+struct fh_dit;
+int fh_dit_probe_wait_timeout(struct fh_dit* m, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
