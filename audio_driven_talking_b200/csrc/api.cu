@@ -72,7 +72,9 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, 
 inline size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-int bn_for(int N) { return (N % 256 == 0 && N >= 4096) ? 256 : 128; }
+// Tile width per GEMM, measured on B200 at 1280 tokens: 256 columns only for the widest
+// (FFN1, cross-KV); 128 for QKV (better waves over 148 SMs) and the width-1536 GEMMs.
+int bn_for(int N) { return (N % 256 == 0 && N >= 8192) ? 256 : 128; }
 
 struct TensorRec {
   int tid;

@@ -92,7 +92,6 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  pdl_launch_dependents();
   if (warp == 0) {
     if (lane == 0) {
       // The weights W are never written by any kernel: start streaming the first stages'
@@ -130,6 +129,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     producer_done:
+      pdl_launch_dependents();  // every tile load is issued: the next kernel may start its prologue
       if (*abort_flag) {
         // let every copy this thread started land before the CTA's shared memory goes away;
         // W tiles issued ahead of the dependency wait whose A half never followed cannot

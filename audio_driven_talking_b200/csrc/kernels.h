@@ -13,10 +13,11 @@ namespace fh {
 typedef __nv_bfloat16 bf16;
 struct EpiParams;
 
-// Launch helper. Every kernel of this library calls pdl_wait() before it touches global
-// memory an earlier kernel writes, so launches may set programmatic stream serialization
-// (PDL); measured on B200 with the trigger at kernel entry it cost ~0.9 ms per slice, so
-// the attribute is not set and the kernel-side hooks are no-ops.
+// Launch with programmatic stream serialization (PDL): a kernel may begin its prologue
+// while its predecessor in the stream drains. Every kernel of this library calls
+// pdl_wait() before it touches global memory that an earlier kernel writes. The GEMM
+// signals its dependents only after its producer has issued the last tile loads (a
+// trigger at kernel entry measured slower on B200: the early dependents took SM slots).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                               Args&&... args) {
@@ -25,8 +26,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
