@@ -72,9 +72,23 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, 
 inline size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Tile width per GEMM, measured on B200 at 1280 tokens: 256 columns only for the widest
-// (FFN1, cross-KV); 128 for QKV (better waves over 148 SMs) and the width-1536 GEMMs.
-int bn_for(int N) { return (N % 256 == 0 && N >= 8192) ? 256 : 128; }
+// Tile shape per GEMM, from the weight's N and K. Deep projections (K >= 1024, N >= 1536:
+// QKV, O-proj, cross-Q/O, FFN1, FFN2) run as 256-row tiles on CTA pairs (cta_group::2),
+// each CTA streaming half of the W tile; the rest (patch embed K=256, head N=128, the
+// per-slice cross-KV with 160 rows) on single CTAs. Tile width 256 only for the widest
+// (FFN1, cross-KV); 128 elsewhere (measured on B200 at 1280 tokens).
+struct TileCfg {
+  int bn;
+  bool pair;
+  int wbox;  // rows of the W tile each CTA loads
+};
+TileCfg tile_cfg(int N, int K, bool pair_ok = true) {
+  TileCfg t;
+  t.bn = (N % 256 == 0 && N >= 8192) ? 256 : 128;
+  t.pair = pair_ok && K >= 1024 && N >= 1536 && N <= 16384;
+  t.wbox = t.pair ? t.bn / 2 : t.bn;
+  return t;
+}
 
 struct TensorRec {
   int tid;
@@ -242,8 +256,10 @@ int run_gemm(fh_dit* m, const CUtensorMap* amap, const void* A, long lda, const 
              int tclass) {
   const int ti = timed_begin(m, tclass, st);
   cudaError_t e;
-  if (m->bf16)
-    e = gemm_tc(*amap, *bmap, M, N, K, bn_for(N), kind, out_bf16, ep, m->err_dev, m->num_sms, st);
+  if (m->bf16) {
+    const TileCfg tc = tile_cfg(N, K);
+    e = gemm_tc(*amap, *bmap, M, N, K, tc.bn, kind, out_bf16, ep, m->err_dev, m->num_sms, st, tc.pair);
+  }
   else
     e = gemm_simt(reinterpret_cast<const float*>(A), lda, reinterpret_cast<const float*>(W), ldw, M, N, K, kind,
                   ep, st);
@@ -716,13 +732,15 @@ int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** ou
     bool ok = true;
     for (long k = 0; k < NB && ok; ++k) {
       BlockW& b = m->blk[k];
-      ok = make_map(&b.m_qkv, b.wqkv, 3 * D, D, bn_for(3 * D)) && make_map(&b.m_o, b.wo, D, D, bn_for(D)) &&
-           make_map(&b.m_cq, b.wcq, D, D, bn_for(D)) && make_map(&b.m_co, b.wco, D, D, bn_for(D)) &&
-           make_map(&b.m_1, b.w1, FF, D, bn_for(FF)) && make_map(&b.m_2, b.w2, D, FF, bn_for(D)) &&
-           make_map(&b.m_ckv, (uint8_t*)m->wckv + (size_t)k * 2 * D * D * e, 2 * D, D, bn_for(2 * D));
+      auto box = [](long n, long kk) { return (uint32_t)tile_cfg((int)n, (int)kk).wbox; };
+      ok = make_map(&b.m_qkv, b.wqkv, 3 * D, D, box(3 * D, D)) && make_map(&b.m_o, b.wo, D, D, box(D, D)) &&
+           make_map(&b.m_cq, b.wcq, D, D, box(D, D)) && make_map(&b.m_co, b.wco, D, D, box(D, D)) &&
+           make_map(&b.m_1, b.w1, FF, D, box(FF, D)) && make_map(&b.m_2, b.w2, D, FF, box(D, FF)) &&
+           make_map(&b.m_ckv, (uint8_t*)m->wckv + (size_t)k * 2 * D * D * e, 2 * D, D, box(2 * D, D));
     }
-    ok = ok && make_map(&m->m_ckv_all, m->wckv, NB * 2 * D, D, bn_for(NB * 2 * D)) &&
-         make_map(&m->m_patch, m->patch_w, D, 2 * C, bn_for(D)) && make_map(&m->m_head, m->head_w, C, D, bn_for(C));
+    auto box = [](long n, long kk) { return (uint32_t)tile_cfg((int)n, (int)kk).wbox; };
+    ok = ok && make_map(&m->m_ckv_all, m->wckv, NB * 2 * D, D, box(NB * 2 * D, D)) &&
+         make_map(&m->m_patch, m->patch_w, D, 2 * C, box(D, 2 * C)) && make_map(&m->m_head, m->head_w, C, D, box(C, D));
     if (!ok) rc = fail(FH_ERR_CUDA, "weight tensor map encoding failed");
   }
   if (rc == FH_OK) {
@@ -1005,14 +1023,15 @@ int fh_op_linear(const void* A, const void* W, const float* bias, float* out, in
   if (dtype == FH_BF16) {
     if (K % 64) return fail(FH_ERR_SHAPE, "K %% 64 != 0");
     if (!load_encode()) return fail(FH_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled unavailable");
-    const int bn = bn_for(N);
+    const TileCfg tc = tile_cfg(N, K);
     CUtensorMap ma, mb;
-    if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, W, N, K, bn)) return fail(FH_ERR_CUDA, "tensor map encoding");
+    if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, W, N, K, tc.wbox))
+      return fail(FH_ERR_CUDA, "tensor map encoding");
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     RUN(prepare_device(dev));
-    e = gemm_tc(ma, mb, M, N, K, bn, EPI_STORE, false, ep, nullptr, sms, st);
+    e = gemm_tc(ma, mb, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, tc.pair);
   } else if (dtype == FH_F32) {
     if (K % 32) return fail(FH_ERR_SHAPE, "K %% 32 != 0");
     e = gemm_simt((const float*)A, K, (const float*)W, K, M, N, K, EPI_STORE, ep, st);

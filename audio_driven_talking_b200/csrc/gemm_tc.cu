@@ -250,6 +250,229 @@ cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, 
   return launch_pdl(gemm_tc_kernel<BN, KIND, OutT>, dim3(grid), dim3(192), S::SMEM, st, a, b, M, N, K, ep, err);
 }
 
+
+// ------------------------------------------------------------------ CTA-pair variant
+// Two CTAs of a cluster compute a 256 x BN tile with tcgen05.mma.cta_group::2: each CTA
+// loads its own 128 rows of A and half (BN/2 rows) of the W tile, the even CTA issues
+// M=256 MMAs that read both CTAs' shared memory, and each CTA's TMEM receives its 128
+// rows. Per unit of MMA work a CTA streams A + W/2 instead of A + W, which is what the
+// per-SM operand bandwidth limits at these sizes. All loads are per-CTA (no multicast).
+template <int BN>
+struct Tc2Shape {
+  static constexpr int BNH = BN / 2;
+  static constexpr int STAGES = (BN == 256) ? 6 : 8;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BNH * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr uint32_t TX_BYTES = 2 * STAGE_BYTES;  // both CTAs' loads complete on the even CTA's barrier
+  static constexpr uint32_t SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+};
+
+template <int BN, int KIND, typename OutT>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
+                    int K, EpiParams ep, unsigned* err) {
+  using S = Tc2Shape<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::STAGES * S::STAGE_BYTES);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* tfull = empty + S::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* dealloc_bar = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(dealloc_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: the CTA that issues the pair's MMAs
+  const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const int num_m = (M + 2 * BM - 1) / (2 * BM);
+  const int num_n = N / BN;
+  const int ntiles = num_m * num_n;
+  const int nk = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * 128);  // both CTAs' epilogue threads
+    }
+    mbar_init(dealloc_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, 2 * BN);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = cl; tile < ntiles; tile += ncl) {
+        const int m0 = (tile % num_m) * 2 * BM + (int)rank * BM;
+        const int n0 = (tile / num_m) * BN + (int)rank * S::BNH;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) goto producer_done;
+          uint8_t* sa = smem + stage * S::STAGE_BYTES;
+          if (rank == 0) mbar_expect_tx(&full[stage], S::TX_BYTES);
+          const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+          tma_load_2d_pair(&tmA, bar0, sa, kb * BK, m0);
+          tma_load_2d_pair(&tmB, bar0, sa + S::A_BYTES, kb * BK, n0);
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    producer_done:
+      pdl_launch_dependents();
+      if (*abort_flag) {  // give copies already issued time to land (their barrier is the even CTA's)
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      for (int tile = cl; tile < ntiles; tile += ncl, ++local) {
+        const int acc = local & 1;
+        const uint32_t aph = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + S::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_f16_pair(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32), idesc,
+                            (kb | k) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[stage], 0x3);
+          if (++stage == S::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair(&tfull[acc], 0x3);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    pdl_wait();
+    int local = 0;
+    for (int tile = cl; tile < ntiles; tile += ncl, ++local) {
+      const int acc = local & 1;
+      const uint32_t aph = (local >> 1) & 1;
+      const int m0 = (tile % num_m) * 2 * BM + (int)rank * BM;
+      const int n0 = (tile / num_m) * BN;
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      if constexpr (KIND == EPI_RESID && BN == 128) {
+        float4 xr[32];
+        const float4* xrow = reinterpret_cast<const float4*>(ep.resid + (long)(row < M ? row : 0) * ep.ldr + n0);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) xr[i] = xrow[i];
+        bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) {
+          float v[32];
+          tmem_ld32(tb + c, v);
+          tc_wait_ld();
+          if (row < M) epi_resid_chunk_pref(ep, row, n0 + c, v, &xr[c >> 2]);
+        }
+      } else {
+        bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int g = 0; g < BN; g += 128) {
+          float ssq = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            float v[32];
+            tmem_ld32(tb + g + c, v);
+            tc_wait_ld();
+            if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
+          }
+          if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    // both CTAs are past their last TMEM access before the pair's allocation is released
+    if (lane == 0) {
+      mbar_arrive_cluster(mapa_shared(smem_u32(dealloc_bar), rank ^ 1u));
+      drain_wait(dealloc_bar, 0);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, 2 * BN);
+  }
+}
+
+template <int BN, int KIND, typename OutT>
+cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, const EpiParams& ep,
+                       unsigned* err, int num_sms, cudaStream_t st) {
+  using S = Tc2Shape<BN>;
+  const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
+  int clusters = num_sms / 2;
+  if (tiles < clusters) clusters = tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = S::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, KIND, OutT>, a, b, M, N, K, ep, err);
+}
+
+template <int BN, int KIND, typename OutT>
+cudaError_t prepare_tc2() {
+  return cudaFuncSetAttribute(gemm_tc2_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Tc2Shape<BN>::SMEM);
+}
+
 template <int BN, int KIND, typename OutT>
 cudaError_t prepare_tc() {
   return cudaFuncSetAttribute(gemm_tc_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -263,16 +486,23 @@ cudaError_t gemm_tc_prepare() {
       prepare_tc<128, EPI_STORE, bf16>(), prepare_tc<256, EPI_STORE, bf16>(), prepare_tc<128, EPI_GELU, bf16>(),
       prepare_tc<256, EPI_GELU, bf16>(),  prepare_tc<128, EPI_NORM, bf16>(),  prepare_tc<256, EPI_NORM, bf16>(),
       prepare_tc<128, EPI_QKV, bf16>(),   prepare_tc<256, EPI_QKV, bf16>(),   prepare_tc<128, EPI_RESID, bf16>(),
-      prepare_tc<256, EPI_RESID, bf16>(), prepare_tc<128, EPI_STORE, float>(), prepare_tc<256, EPI_STORE, float>()};
+      prepare_tc<256, EPI_RESID, bf16>(), prepare_tc<128, EPI_STORE, float>(), prepare_tc<256, EPI_STORE, float>(),
+      prepare_tc2<128, EPI_STORE, bf16>(), prepare_tc2<256, EPI_STORE, bf16>(), prepare_tc2<128, EPI_GELU, bf16>(),
+      prepare_tc2<256, EPI_GELU, bf16>(), prepare_tc2<128, EPI_NORM, bf16>(), prepare_tc2<256, EPI_NORM, bf16>(),
+      prepare_tc2<128, EPI_QKV, bf16>(), prepare_tc2<256, EPI_QKV, bf16>(), prepare_tc2<128, EPI_RESID, bf16>(),
+      prepare_tc2<256, EPI_RESID, bf16>(), prepare_tc2<128, EPI_STORE, float>(),
+      prepare_tc2<256, EPI_STORE, float>()};
   for (cudaError_t e : es)
     if (e != cudaSuccess) return e;
   return cudaSuccess;
 }
 
 cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int bn, int kind,
-                    bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st) {
-#define FH_TC_CASE(BNV, KV, OT)                                          \
-  if (bn == BNV && kind == KV) return launch_tc<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st);
+                    bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st, bool pair) {
+#define FH_TC_CASE(BNV, KV, OT)                                                                     \
+  if (bn == BNV && kind == KV)                                                                      \
+    return pair ? launch_tc2<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st)                      \
+                : launch_tc<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st);
   if (out_bf16) {
     FH_TC_CASE(128, EPI_STORE, bf16)
     FH_TC_CASE(256, EPI_STORE, bf16)

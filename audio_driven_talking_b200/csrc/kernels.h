@@ -35,11 +35,13 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 // bf16 tensor-core GEMM (gemm_tc.cu): out = epilogue(A[M,K] * W[N,K]^T); `a`, `b`
-// are TMA maps of A (box 64 x 128) and W (box 64 x bn) with the 128-byte swizzle.
-// N % bn == 0, K % 64 == 0.
+// are TMA maps of A (box 64 x 128) and W (box 64 x bn, or 64 x bn/2 when `pair`) with
+// the 128-byte swizzle. N % bn == 0, K % 64 == 0. `pair`: 256 x bn tiles computed by
+// two CTAs of a cluster with cta_group::2.
 cudaError_t gemm_tc_prepare();  // sets the kernels' shared-memory attributes on the current device
 cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int bn, int kind,
-                    bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st);
+                    bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
+                    bool pair = false);
 
 // fp32 CUDA-core GEMM (misc.cu) with the same epilogues; N % 128 == 0.
 cudaError_t gemm_simt(const float* A, long lda, const float* W, long ldw, int M, int N, int K, int kind,

@@ -25,8 +25,10 @@ def _bf16_operands(seed, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (160, 256, 1536), (300, 1536, 256), (1280, 1536, 1536),
-                                   (1280, 4608, 1536), (1280, 1536, 8960), (8640, 8960, 1536), (1, 128, 128)])
+                                   (1280, 4608, 1536), (1280, 1536, 8960), (8640, 8960, 1536), (1, 128, 128),
+                                   (300, 1536, 1024), (1280, 8960, 1536)])
 def test_linear_bf16_tensor_core(M, N, K):
+    """Single-CTA tiles, and 256-row CTA-pair tiles (cta_group::2) for K >= 1024, N >= 1536."""
     A, W, b = _bf16_operands(M + N + K, M, N, K)
     out = fh.linear(to_dev(A, torch.bfloat16), to_dev(W, torch.bfloat16), to_dev(b))
     torch.cuda.synchronize()
