@@ -156,6 +156,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           if (!load_v(j)) break;
         }
       }
+      // tail: the MMA's release commits for the last K and V tiles have landed
+      for (int j = kiss - 2 < 0 ? 0 : kiss - 2; !*abort_flag && j < kiss; ++j)
+        mbar_wait(&k_empty[j & 1], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+      for (int j = viss - 2 < 0 ? 0 : viss - 2; !*abort_flag && j < viss; ++j)
+        mbar_wait(&v_empty[j & 1], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       if (*abort_flag) {
         uint64_t t0 = globaltimer();
         while (!mbar_try_wait(q_full, 0) && globaltimer() - t0 < FH_WAIT_LIMIT_NS) {

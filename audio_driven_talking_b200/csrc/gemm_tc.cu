@@ -130,6 +130,19 @@ __global__ void __launch_bounds__(192, 1)
       }
     producer_done:
       pdl_launch_dependents();  // every tile load is issued: the next kernel may start its prologue
+      // tail: wait until the MMA has released the stages filled last, so no commit arrival
+      // is still in flight towards this CTA's barriers when it exits
+      if (!*abort_flag) {
+        for (int s = 0; s < S::STAGES && s < issues; ++s) {
+          int st = stage - 1 - s;
+          uint32_t ph = phase;
+          if (st < 0) {
+            st += S::STAGES;
+            ph ^= 1u;
+          }
+          mbar_wait(&empty[st], ph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+        }
+      }
       if (*abort_flag) {
         // let every copy this thread started land before the CTA's shared memory goes away;
         // W tiles issued ahead of the dependency wait whose A half never followed cannot
@@ -182,6 +195,11 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (!ok) break;
         tc_commit(&tfull[acc]);
+      }
+      // tail: the epilogue has released the last accumulators (no arrival left in flight)
+      for (int i = 0; i < 2 && i < local; ++i) {
+        const int t = local - 1 - i;
+        if (!mbar_wait(&tempty[t & 1], (t >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) break;
       }
     }
   } else {
@@ -321,6 +339,7 @@ __global__ void __launch_bounds__(192, 1)
       pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
+      int issues = 0;
       for (int tile = cl; tile < ntiles; tile += ncl) {
         const int m0 = (tile % num_m) * 2 * BM + (int)rank * BM;
         const int n0 = (tile / num_m) * BN + (int)rank * S::BNH;
@@ -331,6 +350,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
           tma_load_2d_pair(&tmA, bar0, sa, kb * BK, m0);
           tma_load_2d_pair(&tmB, bar0, sa + S::A_BYTES, kb * BK, n0);
+          ++issues;
           if (++stage == S::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -339,6 +359,19 @@ __global__ void __launch_bounds__(192, 1)
       }
     producer_done:
       pdl_launch_dependents();
+      // tail: the even CTA's MMA has released (multicast commit into this CTA) every stage
+      // filled last, so no arrival is in flight towards this CTA when it exits
+      if (!*abort_flag) {
+        for (int s = 0; s < S::STAGES && s < issues; ++s) {
+          int st = stage - 1 - s;
+          uint32_t ph = phase;
+          if (st < 0) {
+            st += S::STAGES;
+            ph ^= 1u;
+          }
+          mbar_wait(&empty[st], ph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+        }
+      }
       if (*abort_flag) {  // give copies already issued time to land (their barrier is the even CTA's)
         const uint64_t t0 = globaltimer();
         while (globaltimer() - t0 < 200000ull) {
@@ -379,6 +412,12 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (!ok) break;
         tc_commit_pair(&tfull[acc], 0x3);
+      }
+      // tail: both CTAs' epilogues have released the last accumulators (their arrivals,
+      // local and remote, have landed on this CTA's barriers)
+      for (int i = 0; i < 2 && i < local; ++i) {
+        const int t = local - 1 - i;
+        if (!mbar_wait(&tempty[t & 1], (t >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) break;
       }
     }
   } else {

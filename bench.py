@@ -54,8 +54,8 @@ def slice_tflop() -> float:
 
 
 # launches per class inside one slice, and each launch's algorithmic flops
-CLASS_NAMES = {1: "gemm_tc_kernel<128,EPI_RESID> (O-proj, cross-O, FFN2 with gated residual)",
-               2: "gemm_tc_kernel<256,EPI_GELU> (FFN1)"}
+CLASS_NAMES = {1: "gemm_tc2_kernel<128,EPI_RESID> (CTA pair; O-proj, cross-O, FFN2 with gated residual)",
+               2: "gemm_tc2_kernel<256,EPI_GELU> (CTA pair; FFN1)"}
 
 
 def class_flops_per_launch(cls: int) -> float:
