@@ -69,6 +69,27 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, 
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D view [rows, cols] with row pitch `ld` elements for the GEMM epilogue's TMA stores:
+// box 32 x 32, fp32 with the 128-byte swizzle or bf16 with the 64-byte swizzle.
+bool make_out_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, bool f32) {
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * es};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// output map of a CTA-pair GEMM epilogue (null for the head-major q/k/v scatter)
+bool epi_out_map(CUtensorMap* map, int kind, bool out_bf16, const EpiParams& ep, int M, int N) {
+  if (kind == EPI_QKV) return true;
+  if (kind == EPI_RESID) return make_out_map(map, ep.resid, M, N, ep.ldr, true);
+  return make_out_map(map, ep.out, M, N, ep.ldo, !out_bf16);
+}
+
 inline size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -258,7 +279,13 @@ int run_gemm(fh_dit* m, const CUtensorMap* amap, const void* A, long lda, const 
   cudaError_t e;
   if (m->bf16) {
     const TileCfg tc = tile_cfg(N, K);
-    e = gemm_tc(*amap, *bmap, M, N, K, tc.bn, kind, out_bf16, ep, m->err_dev, m->num_sms, st, tc.pair);
+    CUtensorMap cmap;
+    if (tc.pair && !epi_out_map(&cmap, kind, out_bf16, ep, M, N)) {
+      timed_end(m, ti, st);
+      return fail(FH_ERR_CUDA, "tensor map encoding failed for a GEMM output");
+    }
+    e = gemm_tc(*amap, *bmap, tc.pair && kind != EPI_QKV ? &cmap : nullptr, M, N, K, tc.bn, kind, out_bf16, ep,
+                m->err_dev, m->num_sms, st, tc.pair);
   }
   else
     e = gemm_simt(reinterpret_cast<const float*>(A), lda, reinterpret_cast<const float*>(W), ldw, M, N, K, kind,
@@ -1024,14 +1051,15 @@ int fh_op_linear(const void* A, const void* W, const float* bias, float* out, in
     if (K % 64) return fail(FH_ERR_SHAPE, "K %% 64 != 0");
     if (!load_encode()) return fail(FH_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled unavailable");
     const TileCfg tc = tile_cfg(N, K);
-    CUtensorMap ma, mb;
-    if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, W, N, K, tc.wbox))
+    CUtensorMap ma, mb, mc;
+    if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, W, N, K, tc.wbox) ||
+        !make_out_map(&mc, out, M, N, N, true))
       return fail(FH_ERR_CUDA, "tensor map encoding");
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     RUN(prepare_device(dev));
-    e = gemm_tc(ma, mb, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, tc.pair);
+    e = gemm_tc(ma, mb, &mc, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, tc.pair);
   } else if (dtype == FH_F32) {
     if (K % 32) return fail(FH_ERR_SHAPE, "K %% 32 != 0");
     e = gemm_simt((const float*)A, K, (const float*)W, K, M, N, K, EPI_STORE, ep, st);

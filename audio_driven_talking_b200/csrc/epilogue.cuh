@@ -47,25 +47,22 @@ __device__ __forceinline__ bool epi_normed(const EpiParams& p, int col) {
   return (col % p.norm_period) < p.norm_count;
 }
 
-template <int KIND, typename OutT>
-__device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0, float (&v)[32],
-                                          float& ssq_acc) {
+// The arithmetic of the epilogue on 32 consecutive columns of one row, in registers:
+//   EPI_STORE  v = acc + bias;   EPI_GELU  v = gelu_tanh(acc + bias)
+//   EPI_RESID  v = gate * (acc + bias)  (the increment of the residual)
+//   EPI_NORM / EPI_QKV  v = acc + bias; on normed columns ssq_acc += sum v^2 and v *= gain
+template <int KIND>
+__device__ __forceinline__ void epi_math(const EpiParams& p, int row, int col0, float (&v)[32], float& ssq_acc) {
   const float* b = p.bias + col0;
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
     float4 bb = *reinterpret_cast<const float4*>(b + j);
     v[j] += bb.x; v[j + 1] += bb.y; v[j + 2] += bb.z; v[j + 3] += bb.w;
   }
-  if constexpr (KIND == EPI_STORE || KIND == EPI_GELU) {
-    if constexpr (KIND == EPI_GELU) {
+  if constexpr (KIND == EPI_GELU) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
-    }
-    OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)row * p.ldo + col0;
-#pragma unroll
-    for (int j = 0; j < 32; j += 8) store8(dst + j, v + j);
+    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
   } else if constexpr (KIND == EPI_RESID) {
-    float* r = p.resid + (long)row * p.ldr + col0;
     if (p.gate) {
       const float* g = p.gate + (long)(row / p.rows_per_batch) * p.gate_bstride + col0;
 #pragma unroll
@@ -74,15 +71,8 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0,
         v[j] *= gg.x; v[j + 1] *= gg.y; v[j + 2] *= gg.z; v[j + 3] *= gg.w;
       }
     }
-#pragma unroll
-    for (int j = 0; j < 32; j += 4) {
-      float4 x = *reinterpret_cast<float4*>(r + j);
-      x.x += v[j]; x.y += v[j + 1]; x.z += v[j + 2]; x.w += v[j + 3];
-      *reinterpret_cast<float4*>(r + j) = x;
-    }
-  } else {  // EPI_NORM, EPI_QKV
-    const bool normed = epi_normed(p, col0);
-    if (normed) {
+  } else if constexpr (KIND == EPI_NORM || KIND == EPI_QKV) {
+    if (epi_normed(p, col0)) {
       float s = 0.f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) s = fmaf(v[j], v[j], s);
@@ -94,6 +84,29 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0,
         v[j] *= gg.x; v[j + 1] *= gg.y; v[j + 2] *= gg.z; v[j + 3] *= gg.w;
       }
     }
+  }
+}
+
+// epi_math plus the store by the owning thread (row-major outputs, the residual update,
+// or the head-major q/k/v scatter with rotary).
+template <int KIND, typename OutT>
+__device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0, float (&v)[32],
+                                          float& ssq_acc) {
+  epi_math<KIND>(p, row, col0, v, ssq_acc);
+  if constexpr (KIND == EPI_STORE || KIND == EPI_GELU) {
+    OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)row * p.ldo + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 8) store8(dst + j, v + j);
+  } else if constexpr (KIND == EPI_RESID) {
+    float* r = p.resid + (long)row * p.ldr + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      float4 x = *reinterpret_cast<float4*>(r + j);
+      x.x += v[j]; x.y += v[j + 1]; x.z += v[j + 2]; x.w += v[j + 3];
+      *reinterpret_cast<float4*>(r + j) = x;
+    }
+  } else {  // EPI_NORM, EPI_QKV
+    const bool normed = epi_normed(p, col0);
     if constexpr (KIND == EPI_NORM) {
       OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)row * p.ldo + col0;
 #pragma unroll
@@ -143,6 +156,22 @@ __device__ __forceinline__ void epi_resid_chunk_pref(const EpiParams& p, int row
     x.x += a.x; x.y += a.y; x.z += a.z; x.w += a.w;
     *reinterpret_cast<float4*>(r + j) = x;
   }
+}
+
+// Row `r` (0..31) of a 32-row staging box for a TMA store: 32 values, fp32 rows of 128 bytes
+// in the 128-byte swizzle or bf16 rows of 64 bytes in the 64-byte swizzle (16-byte chunk
+// index XOR address bits 7-9 resp. 7-8), so the 32 lanes' chunks spread over all banks.
+// `box` is aligned to 1024 bytes.
+__device__ __forceinline__ void stage_row(uint8_t* box, int r, const float (&v)[32], float*) {
+  uint8_t* row = box + r * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4*>(row + ((j ^ (r & 7)) << 4)) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+}
+__device__ __forceinline__ void stage_row(uint8_t* box, int r, const float (&v)[32], bf16*) {
+  uint8_t* row = box + r * 64;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) store8(reinterpret_cast<bf16*>(row + ((j ^ ((r >> 1) & 3)) << 4)), v + 8 * j);
 }
 
 template <int KIND>

@@ -20,6 +20,7 @@
 // Every wait is bounded (FH_WAIT_LIMIT_NS); on expiry the CTA latches an error
 // bit, lets the producer's in-flight copies land, frees TMEM and exits.
 #include <cstdio>
+#include <type_traits>
 
 #include "epilogue.cuh"
 #include "kernels.h"
@@ -283,17 +284,24 @@ struct Tc2Shape {
   static constexpr uint32_t B_BYTES = BNH * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr uint32_t TX_BYTES = 2 * STAGE_BYTES;  // both CTAs' loads complete on the even CTA's barrier
-  static constexpr uint32_t SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES;
+  // epilogue staging: per epilogue warp two 32-row boxes of up to 128-byte rows
+  static constexpr uint32_t STG_BYTES = 4 * 2 * 4096;
+  static constexpr uint32_t SMEM = RING_BYTES + STG_BYTES + 1024 /*align*/ + 512 /*barriers*/;
 };
 
 template <int BN, int KIND, typename OutT>
 __global__ void __launch_bounds__(192, 1)
-    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
-                    int K, EpiParams ep, unsigned* err) {
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep, unsigned* err) {
   using S = Tc2Shape<BN>;
+  // every epilogue but the head-major q/k/v scatter leaves through shared memory and TMA
+  constexpr bool STAGED = KIND != EPI_QKV;
+  // element type of the staged boxes: the fp32 residual for EPI_RESID, else the output type
+  using StageT = typename std::conditional<KIND == EPI_RESID, float, OutT>::type;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::STAGES * S::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES + S::STG_BYTES);
   uint64_t* empty = full + S::STAGES;
   uint64_t* tfull = empty + S::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -324,6 +332,7 @@ __global__ void __launch_bounds__(192, 1)
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (STAGED) prefetch_tmap(&tmC);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, 2 * BN);
@@ -422,6 +431,8 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     const int quarter = warp & 3;
+    uint8_t* stg = smem + S::RING_BYTES + quarter * 8192;  // this warp's two staging boxes
+    uint32_t nchunk = 0;
     pdl_wait();
     int local = 0;
     for (int tile = cl; tile < ntiles; tile += ncl, ++local) {
@@ -431,20 +442,45 @@ __global__ void __launch_bounds__(192, 1)
       const int n0 = (tile / num_m) * BN;
       const int row = m0 + quarter * 32 + lane;
       const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      if constexpr (KIND == EPI_RESID && BN == 128) {
-        float4 xr[32];
-        const float4* xrow = reinterpret_cast<const float4*>(ep.resid + (long)(row < M ? row : 0) * ep.ldr + n0);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) xr[i] = xrow[i];
+      if constexpr (STAGED) {
+        // 32 x 32 boxes: this warp's 32 rows, 32 columns at a time, through two staging
+        // buffers; lane 0 issues the TMA store (the residual: an fp32 add in L2)
+        const int row0 = m0 + quarter * 32;
         bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
+#pragma unroll 1
+        for (int g = 0; row0 < M && g < BN; g += 128) {  // a warp with no row below M stores nothing
+          float ssq = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            float v[32];
+            tmem_ld32(tb + g + c, v);
+            tc_wait_ld();
+            if (row < M) {
+              epi_math<KIND>(ep, row, n0 + g + c, v, ssq);
+            } else {
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
-          float v[32];
-          tmem_ld32(tb + c, v);
-          tc_wait_ld();
-          if (row < M) epi_resid_chunk_pref(ep, row, n0 + c, v, &xr[c >> 2]);
+              for (int j = 0; j < 32; ++j) v[j] = 0.f;
+            }
+            // buffers alternate per committed store, so the one group that may still be
+            // reading is the other buffer's
+            uint8_t* box = stg + (nchunk & 1) * 4096;
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            stage_row(box, lane, v, (StageT*)nullptr);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if constexpr (KIND == EPI_RESID)
+                tma_reduce_add_2d(&tmC, box, n0 + g + c, row0);  // rows at or past M are clipped
+              else
+                tma_store_2d(&tmC, box, n0 + g + c, row0);
+              bulk_commit();
+            }
+            ++nchunk;
+          }
+          if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
         }
       } else {
         bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
@@ -466,6 +502,8 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
     }
+    if (STAGED && lane == 0) bulk_wait_all();  // every store issued by this warp has been performed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -483,8 +521,8 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 template <int BN, int KIND, typename OutT>
-cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, const EpiParams& ep,
-                       unsigned* err, int num_sms, cudaStream_t st) {
+cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int M, int N, int K,
+                       const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st) {
   using S = Tc2Shape<BN>;
   const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
   int clusters = num_sms / 2;
@@ -503,7 +541,7 @@ cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, KIND, OutT>, a, b, M, N, K, ep, err);
+  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, KIND, OutT>, a, b, c, M, N, K, ep, err);
 }
 
 template <int BN, int KIND, typename OutT>
@@ -536,11 +574,15 @@ cudaError_t gemm_tc_prepare() {
   return cudaSuccess;
 }
 
-cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K, int bn, int kind,
-                    bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st, bool pair) {
+cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, int M, int N, int K, int bn,
+                    int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
+                    bool pair) {
+  // the CTA-pair kernel stores every epilogue but EPI_QKV through the output map `c`
+  if (pair && kind != EPI_QKV && !c) return cudaErrorInvalidValue;
+  const CUtensorMap& cm = c ? *c : a;
 #define FH_TC_CASE(BNV, KV, OT)                                                                     \
   if (bn == BNV && kind == KV)                                                                      \
-    return pair ? launch_tc2<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st)                      \
+    return pair ? launch_tc2<BNV, KV, OT>(a, b, cm, M, N, K, ep, err, num_sms, st)                  \
                 : launch_tc<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st);
   if (out_bf16) {
     FH_TC_CASE(128, EPI_STORE, bf16)
