@@ -83,9 +83,23 @@ bool make_out_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// output map of a CTA-pair GEMM epilogue (null for the head-major q/k/v scatter)
+// 3D bf16 view of the head-major q/k/v workspace [planes = 3 * B * heads][L][128], box
+// 32 x 32 x 1 with the 64-byte swizzle
+bool make_qkv_map(CUtensorMap* map, const void* base, uint64_t L, uint64_t planes) {
+  cuuint64_t dims[3] = {128, L, planes};
+  cuuint64_t strides[2] = {128 * 2, L * 128 * 2};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// output map of a CTA-pair GEMM epilogue
 bool epi_out_map(CUtensorMap* map, int kind, bool out_bf16, const EpiParams& ep, int M, int N) {
-  if (kind == EPI_QKV) return true;
+  if (kind == EPI_QKV)
+    return out_bf16 && make_qkv_map(map, ep.out, ep.rows_per_batch,
+                                    3ull * (M / ep.rows_per_batch) * (ep.dim >> 7));
   if (kind == EPI_RESID) return make_out_map(map, ep.resid, M, N, ep.ldr, true);
   return make_out_map(map, ep.out, M, N, ep.ldo, !out_bf16);
 }
@@ -284,8 +298,8 @@ int run_gemm(fh_dit* m, const CUtensorMap* amap, const void* A, long lda, const 
       timed_end(m, ti, st);
       return fail(FH_ERR_CUDA, "tensor map encoding failed for a GEMM output");
     }
-    e = gemm_tc(*amap, *bmap, tc.pair && kind != EPI_QKV ? &cmap : nullptr, M, N, K, tc.bn, kind, out_bf16, ep,
-                m->err_dev, m->num_sms, st, tc.pair);
+    e = gemm_tc(*amap, *bmap, tc.pair ? &cmap : nullptr, M, N, K, tc.bn, kind, out_bf16, ep, m->err_dev,
+                m->num_sms, st, tc.pair);
   }
   else
     e = gemm_simt(reinterpret_cast<const float*>(A), lda, reinterpret_cast<const float*>(W), ldw, M, N, K, kind,

@@ -18,6 +18,8 @@
 // the rotation are linear per channel, so RoPE(g * r * y) = r * RoPE(g * y).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace fh {
@@ -51,7 +53,8 @@ __device__ __forceinline__ bool epi_normed(const EpiParams& p, int col) {
 //   EPI_STORE  v = acc + bias;   EPI_GELU  v = gelu_tanh(acc + bias)
 //   EPI_RESID  v = gate * (acc + bias)  (the increment of the residual)
 //   EPI_NORM / EPI_QKV  v = acc + bias; on normed columns ssq_acc += sum v^2 and v *= gain
-template <int KIND>
+// OutT is the type the result is stored in: bf16 results take the hardware tanh in GELU.
+template <int KIND, typename OutT>
 __device__ __forceinline__ void epi_math(const EpiParams& p, int row, int col0, float (&v)[32], float& ssq_acc) {
   const float* b = p.bias + col0;
 #pragma unroll
@@ -60,8 +63,13 @@ __device__ __forceinline__ void epi_math(const EpiParams& p, int row, int col0, 
     v[j] += bb.x; v[j + 1] += bb.y; v[j + 2] += bb.z; v[j + 3] += bb.w;
   }
   if constexpr (KIND == EPI_GELU) {
+    if constexpr (std::is_same<OutT, bf16>::value) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh_approx(v[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_tanh(v[j]);
+    }
   } else if constexpr (KIND == EPI_RESID) {
     if (p.gate) {
       const float* g = p.gate + (long)(row / p.rows_per_batch) * p.gate_bstride + col0;
@@ -87,12 +95,27 @@ __device__ __forceinline__ void epi_math(const EpiParams& p, int row, int col0, 
   }
 }
 
+// EPI_QKV on q and k columns: rotate adjacent pairs (2d, 2d+1) by the angles of the row's
+// token position (table (cos, sin) [rows_per_batch, 64]).
+__device__ __forceinline__ void epi_rope(const EpiParams& p, int row, int col0, float (&v)[32]) {
+  const int l = row % p.rows_per_batch;
+  const int d0 = (col0 % p.dim) & 127;
+  const float2* rt = p.rope + (long)l * 64 + (d0 >> 1);
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    float2 cs = rt[j >> 1];
+    float x0 = v[j], x1 = v[j + 1];
+    v[j] = x0 * cs.x - x1 * cs.y;
+    v[j + 1] = x0 * cs.y + x1 * cs.x;
+  }
+}
+
 // epi_math plus the store by the owning thread (row-major outputs, the residual update,
 // or the head-major q/k/v scatter with rotary).
 template <int KIND, typename OutT>
 __device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0, float (&v)[32],
                                           float& ssq_acc) {
-  epi_math<KIND>(p, row, col0, v, ssq_acc);
+  epi_math<KIND, OutT>(p, row, col0, v, ssq_acc);
   if constexpr (KIND == EPI_STORE || KIND == EPI_GELU) {
     OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)row * p.ldo + col0;
 #pragma unroll
@@ -118,16 +141,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0,
       const int cin = col0 - sec * p.dim;
       const int head = cin >> 7;
       const int d0 = cin & 127;
-      if (normed) {
-        const float2* rt = p.rope + (long)l * 64 + (d0 >> 1);
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          float2 cs = rt[j >> 1];
-          float x0 = v[j], x1 = v[j + 1];
-          v[j] = x0 * cs.x - x1 * cs.y;
-          v[j + 1] = x0 * cs.y + x1 * cs.x;
-        }
-      }
+      if (normed) epi_rope(p, row, col0, v);
       const int heads = p.dim >> 7;
       OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)sec * p.sec_stride +
                   (((long)bidx * heads + head) * p.rows_per_batch + l) * 128 + d0;

@@ -295,8 +295,9 @@ __global__ void __launch_bounds__(192, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep, unsigned* err) {
   using S = Tc2Shape<BN>;
-  // every epilogue but the head-major q/k/v scatter leaves through shared memory and TMA
-  constexpr bool STAGED = KIND != EPI_QKV;
+  // every epilogue leaves through shared memory and TMA stores (EPI_QKV: a 3D map over the
+  // head-major [3 * B * heads][L][128] layout, except for warps whose rows cross a stream)
+  constexpr bool STAGED = true;
   // element type of the staged boxes: the fp32 residual for EPI_RESID, else the output type
   using StageT = typename std::conditional<KIND == EPI_RESID, float, OutT>::type;
   extern __shared__ uint8_t smem_raw[];
@@ -449,6 +450,15 @@ __global__ void __launch_bounds__(192, 1)
         bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
+        // EPI_QKV: the 32 rows stay inside one stream (row0 and L both multiples of 32 at
+        // the usual sizes); otherwise this warp stores directly, row by row
+        bool direct = false;
+        int l0 = 0, bidx = 0;
+        if constexpr (KIND == EPI_QKV) {
+          l0 = row0 % ep.rows_per_batch;
+          bidx = row0 / ep.rows_per_batch;
+          direct = l0 + 32 > ep.rows_per_batch && row0 + (ep.rows_per_batch - l0) < M;
+        }
 #pragma unroll 1
         for (int g = 0; row0 < M && g < BN; g += 128) {  // a warp with no row below M stores nothing
           float ssq = 0.f;
@@ -457,8 +467,14 @@ __global__ void __launch_bounds__(192, 1)
             float v[32];
             tmem_ld32(tb + g + c, v);
             tc_wait_ld();
+            if (direct) {
+              if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
+              continue;
+            }
             if (row < M) {
-              epi_math<KIND>(ep, row, n0 + g + c, v, ssq);
+              epi_math<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
+              if constexpr (KIND == EPI_QKV)
+                if (epi_normed(ep, n0 + g + c)) epi_rope(ep, row, n0 + g + c, v);
             } else {
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -472,10 +488,17 @@ __global__ void __launch_bounds__(192, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              if constexpr (KIND == EPI_RESID)
-                tma_reduce_add_2d(&tmC, box, n0 + g + c, row0);  // rows at or past M are clipped
-              else
-                tma_store_2d(&tmC, box, n0 + g + c, row0);
+              const int col = n0 + g + c;
+              if constexpr (KIND == EPI_RESID) {
+                tma_reduce_add_2d(&tmC, box, col, row0);  // rows at or past M are clipped
+              } else if constexpr (KIND == EPI_QKV) {
+                const int sec = col / ep.dim, cin = col - sec * ep.dim;
+                const int heads = ep.dim >> 7;
+                const int nb = M / ep.rows_per_batch;
+                tma_store_3d(&tmC, box, cin & 127, l0, (sec * nb + bidx) * heads + (cin >> 7));
+              } else {
+                tma_store_2d(&tmC, box, col, row0);
+              }
               bulk_commit();
             }
             ++nchunk;
@@ -577,8 +600,8 @@ cudaError_t gemm_tc_prepare() {
 cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, int M, int N, int K, int bn,
                     int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
                     bool pair) {
-  // the CTA-pair kernel stores every epilogue but EPI_QKV through the output map `c`
-  if (pair && kind != EPI_QKV && !c) return cudaErrorInvalidValue;
+  // the CTA-pair kernel stores its epilogue through the output map `c`
+  if (pair && !c) return cudaErrorInvalidValue;
   const CUtensorMap& cm = c ? *c : a;
 #define FH_TC_CASE(BNV, KV, OT)                                                                     \
   if (bn == BNV && kind == KV)                                                                      \

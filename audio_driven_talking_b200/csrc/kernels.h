@@ -37,9 +37,9 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // bf16 tensor-core GEMM (gemm_tc.cu): out = epilogue(A[M,K] * W[N,K]^T); `a`, `b`
 // are TMA maps of A (box 64 x 128) and W (box 64 x bn, or 64 x bn/2 when `pair`) with
 // the 128-byte swizzle. N % bn == 0, K % 64 == 0. `pair`: 256 x bn tiles computed by
-// two CTAs of a cluster with cta_group::2; their epilogues (all but EPI_QKV) store through
-// `c`, a TMA map of the output (EPI_RESID: of the fp32 residual) with box 32 x 32 and the
-// 128-byte (fp32) or 64-byte (bf16) swizzle.
+// two CTAs of a cluster with cta_group::2; their epilogues store through `c`, a TMA map of
+// the output (EPI_RESID: of the fp32 residual; EPI_QKV: 3D [3*B*heads][L][128]) with box
+// 32 x 32 (x 1) and the 128-byte (fp32) or 64-byte (bf16) swizzle.
 cudaError_t gemm_tc_prepare();  // sets the kernels' shared-memory attributes on the current device
 cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, int M, int N, int K, int bn,
                     int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
