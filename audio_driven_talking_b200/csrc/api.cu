@@ -83,6 +83,18 @@ bool make_out_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t co
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D bf16 view [d2][d1][d0] (d0 contiguous), box box0 x box1 x 1, 128-byte swizzle.
+bool make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                 uint32_t box1) {
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * 2, d1 * d0 * 2};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3D bf16 view of the head-major q/k/v workspace [planes = 3 * B * heads][L][128], box
 // 32 x 32 x 1 with the 64-byte swizzle
 bool make_qkv_map(CUtensorMap* map, const void* base, uint64_t L, uint64_t planes) {
@@ -150,6 +162,7 @@ struct Plan {
   int batch = 0;
   WsLayout lay{};
   CUtensorMap m_h, m_attn, m_u, m_tok, m_audio, m_q, m_k, m_v;
+  CUtensorMap m_xq, m_xkv, m_xo;  // cross-attention: queries and output per frame, keys/values
 };
 
 struct GraphEntry {
@@ -262,6 +275,10 @@ int get_plan(fh_dit* m, void* ws, int B, Plan** out) {
     ok = ok && make_map(&p.m_q, at<void>(ws, w.qkv), rows, 128, 128) &&
          make_map(&p.m_k, at<void>(ws, w.qkv + sec), rows, 128, 128) &&
          make_map(&p.m_v, at<void>(ws, w.qkv + 2 * sec), rows, 128, 128);
+    const uint64_t HW = m->L / m->F, frames = (uint64_t)B * m->F;
+    ok = ok && make_map_3d(&p.m_xq, at<void>(ws, w.cq), m->D, HW, frames, 64, 128) &&
+         make_map_3d(&p.m_xo, at<void>(ws, w.attn), m->D, HW, frames, 64, 32) &&
+         make_map(&p.m_xkv, at<void>(ws, w.ckv), frames * m->A, (uint64_t)m->NB * 2 * m->D, 32);
     if (!ok) {
       p.ws = nullptr;
       return fail(FH_ERR_CUDA, "tensor map encoding failed for the workspace");
@@ -451,9 +468,13 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
   }
   {
     const int ti = timed_begin(m, 5, st);
-    cudaError_t e = cross_attn<T>(at<T>(ws, w.cq), at<float>(ws, w.ssq_cq), at<T>(ws, w.ckv), (long)m->NB * 2 * D,
-                                  k * 2 * D, k * 2 * D + D, at<float>(ws, w.ssq_ckv), m->NB * 2 * NH, k * 2 * NH, B,
-                                  NH, L, m->F, m->A, eps, attn, st);
+    cudaError_t e =
+        m->bf16 ? xattn_tc(P.m_xq, P.m_xkv, P.m_xo, at<float>(ws, w.ssq_cq), at<float>(ws, w.ssq_ckv),
+                           m->NB * 2 * NH, k * 2 * NH, k * 2 * D, k * 2 * D + D, B, NH, L, m->F, m->A, eps, m->err_dev,
+                           st)
+                : cross_attn<T>(at<T>(ws, w.cq), at<float>(ws, w.ssq_cq), at<T>(ws, w.ckv), (long)m->NB * 2 * D,
+                                k * 2 * D, k * 2 * D + D, at<float>(ws, w.ssq_ckv), m->NB * 2 * NH, k * 2 * NH, B,
+                                NH, L, m->F, m->A, eps, attn, st);
     timed_end(m, ti, st);
     LAUNCH(e);
   }
@@ -556,6 +577,7 @@ int prepare_device(int dev) {
   cudaError_t e = gemm_tc_prepare();
   if (e == cudaSuccess) e = attn_tc_prepare();
   if (e == cudaSuccess) e = cross_attn_prepare();
+  if (e == cudaSuccess) e = xattn_tc_prepare();
   if (e != cudaSuccess) return fail(FH_ERR_CUDA, "kernel attribute setup: %s", cudaGetErrorString(e));
   if (dev < 32) done |= 1u << dev;
   return FH_OK;

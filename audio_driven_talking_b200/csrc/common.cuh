@@ -84,6 +84,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Wait (bounded, ignoring the abort flag) for a barrier phase that in-flight copies
+// complete, so that shared memory outlives them; false if the limit ran out.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
+  uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > FH_WAIT_LIMIT_NS) return false;
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0,
                                             int c1) {

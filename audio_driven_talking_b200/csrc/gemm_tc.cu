@@ -41,14 +41,6 @@ struct TcShape {
   static constexpr uint32_t SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity) {
-  uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer() - t0 > FH_WAIT_LIMIT_NS) return false;
-  }
-  return true;
-}
-
 template <int BN, int KIND, typename OutT>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,

@@ -63,6 +63,14 @@ cudaError_t attn_simt(const T* q, const T* k, const T* v, const float* ssq, int 
 // q [B*L, D] row-major with ssq_q [B*L, heads]; keys/values: rows (b*F + f)*A + a of
 // kv (row stride ldkv), key columns at koff, value columns at voff, with key partial
 // sums of squares ssq_k[row * ssq_k_ld + ssq_k_off + h]. out [B*L, D].
+// bf16 per-frame cross-attention on the tensor cores (xattn.cu): `q` a 3D TMA map of the
+// cross queries [B*F frames][HW][D] (box 64 x 128 x 1), `kv` a 2D map of the cross
+// keys/values [B*F*A rows][ldkv] (box 64 x 32), `o` a 3D map of the output like `q` with
+// box 64 x 32 x 1; all bf16 with the 128-byte swizzle. A == 32, L % F == 0.
+cudaError_t xattn_tc_prepare();
+cudaError_t xattn_tc(const CUtensorMap& q, const CUtensorMap& kv, const CUtensorMap& o, const float* ssq_q,
+                     const float* ssq_k, int ssq_k_ld, int ssq_k_off, int koff, int voff, int batch, int heads, int L,
+                     int F, int A, float eps, unsigned* err, cudaStream_t st);
 cudaError_t cross_attn_prepare();  // shared-memory attribute, outside any stream capture
 template <typename T>
 cudaError_t cross_attn(const T* q, const float* ssq_q, const T* kv, long ldkv, int koff, int voff,

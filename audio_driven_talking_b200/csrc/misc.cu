@@ -32,6 +32,16 @@ __global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ ou
   float4 v[NV];
 #pragma unroll
   for (int i = 0; i < NV; ++i) v[i] = xr[lane + 32 * i];
+  // the affine / modulation vectors are loaded alongside the row, before the reductions
+  const long mb = (long)(row / rows_per_batch) * mod_bstride;
+  const float* av = mode == 1 ? w : scale + mb;
+  const float* cv = mode == 1 ? bb : shift + mb;
+  float4 ma[NV], mc[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    ma[i] = reinterpret_cast<const float4*>(av)[lane + 32 * i];
+    mc[i] = reinterpret_cast<const float4*>(cv)[lane + 32 * i];
+  }
   float mu = 0.f, rstd;
   if (mode != 2) {
     float s = 0.f;
@@ -51,19 +61,14 @@ __global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ ou
     for (int i = 0; i < NV; ++i) q += (v[i].x * v[i].x + v[i].y * v[i].y) + (v[i].z * v[i].z + v[i].w * v[i].w);
     rstd = rsqrtf(warp_sum(q) * (1.f / D) + eps);
   }
-  const long mb = (long)(row / rows_per_batch) * mod_bstride;
   T* orow = out + (long)row * D;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int col = (lane + 32 * i) * 4;
     float y[4] = {(v[i].x - mu) * rstd, (v[i].y - mu) * rstd, (v[i].z - mu) * rstd, (v[i].w - mu) * rstd};
-    float4 a, c;
-    if (mode == 1) {
-      a = *reinterpret_cast<const float4*>(w + col);
-      c = *reinterpret_cast<const float4*>(bb + col);
-    } else {
-      a = *reinterpret_cast<const float4*>(scale + mb + col);
-      c = *reinterpret_cast<const float4*>(shift + mb + col);
+    float4 a = ma[i];
+    const float4 c = mc[i];
+    if (mode != 1) {
       a.x += 1.f; a.y += 1.f; a.z += 1.f; a.w += 1.f;
     }
     y[0] = y[0] * a.x + c.x;
@@ -543,7 +548,7 @@ template <typename T>
 cudaError_t norm_rows(const float* x, T* out, int M, int D, int rows_per_batch, int mode, const float* shift,
                       const float* scale, long mod_bstride, const float* w, const float* bb, float eps,
                       cudaStream_t st) {
-  const int rows_per_cta = 8;
+  const int rows_per_cta = 4;
   dim3 grid((M + rows_per_cta - 1) / rows_per_cta);
 #define FH_NORM_CASE(NVV)                                                                                     \
   case NVV:                                                                                                   \
