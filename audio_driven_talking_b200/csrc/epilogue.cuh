@@ -110,6 +110,25 @@ __device__ __forceinline__ void epi_rope(const EpiParams& p, int row, int col0, 
   }
 }
 
+// Prefetch into L1 the per-column vectors the epilogue of columns [col0, col0 + n) of
+// `row` will read (bias; gate of the row's stream for EPI_RESID; gain for EPI_NORM/QKV),
+// so that their loads, issued after the accumulator is ready, hit L1. One 128-byte line
+// per 32 columns and vector.
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+template <int KIND>
+__device__ __forceinline__ void epi_prefetch(const EpiParams& p, int row, int col0, int n) {
+  for (int c = 0; c < n; c += 32) {
+    prefetch_l1(p.bias + col0 + c);
+    if constexpr (KIND == EPI_RESID) {
+      if (p.gate) prefetch_l1(p.gate + (long)(row / p.rows_per_batch) * p.gate_bstride + col0 + c);
+    } else if constexpr (KIND == EPI_NORM || KIND == EPI_QKV) {
+      if (epi_normed(p, col0 + c)) prefetch_l1(p.gain + col0 + c);
+    }
+  }
+}
+
 // epi_math plus the store by the owning thread (row-major outputs, the residual update,
 // or the head-major q/k/v scatter with rotary).
 template <int KIND, typename OutT>

@@ -439,6 +439,7 @@ __global__ void __launch_bounds__(192, 1)
         // 32 x 32 boxes: this warp's 32 rows, 32 columns at a time, through two staging
         // buffers; lane 0 issues the TMA store (the residual: an fp32 add in L2)
         const int row0 = m0 + quarter * 32;
+        epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0, BN);  // while the MMAs run
         bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
@@ -565,6 +566,271 @@ cudaError_t prepare_tc2() {
                               (int)Tc2Shape<BN>::SMEM);
 }
 
+// ------------------------------------------------------------------ split-K over two CTA pairs
+// GEMMs with few output tiles (M = 1280, N = 1536: 30 tiles of 256 x 256) run one tile per
+// cluster of four CTAs. CTA pair s (cluster ranks 2s, 2s+1) computes the tile over half of
+// the K range with cta_group::2 MMAs into its own TMEM accumulator, on 256-wide tiles whose
+// operand traffic per MMA is the lowest the pair can have. Pair 1's epilogue warps then
+// write their fp32 accumulator rows into pair 0's shared memory (the operand ring, free
+// once pair 0's MMAs are done) and pair 0 adds them to its own, always in that order,
+// before the usual staged epilogue. One tile per cluster: the host launches this only
+// when 4 x tiles CTAs fit on the GPU.
+template <int BN, int KIND, typename OutT>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc2s_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep, unsigned* err) {
+  using S = Tc2Shape<BN>;
+  static_assert(KIND != EPI_QKV, "the head-major scatter runs on the plain pair kernel");
+  static_assert(BN * 512 <= (int)S::RING_BYTES, "the partial accumulator must fit in the operand ring");
+  using StageT = typename std::conditional<KIND == EPI_RESID, float, OutT>::type;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES + S::STG_BYTES);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* tfull = empty + S::STAGES;
+  uint64_t* ring_free = tfull + 1;   // on pair 1: pair 0's ring may be overwritten
+  uint64_t* part_ready = ring_free + 1;  // [4] on pair 0: a quarter's partial rows have landed
+  uint64_t* done = part_ready + 4;   // every other CTA of the cluster is finished with this one
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t split = rank >> 1;      // which half of K
+  const uint32_t half = rank & 1;        // which 128 rows of the tile
+  const uint32_t lead = rank & 2;        // the pair's MMA-issuing CTA
+  const uint16_t mask = (uint16_t)(0x3u << lead);
+  const int tile = blockIdx.x >> 2;
+  const int num_m = (M + 2 * BM - 1) / (2 * BM);
+  const int m0 = (tile % num_m) * 2 * BM + (int)half * BM;
+  const int n0 = (tile / num_m) * BN;
+  const int nk = (K + BK - 1) / BK;
+  const int kb0 = split ? nk / 2 : 0, kb1 = split ? nk : nk / 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(ring_free, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&part_ready[q], 1);
+    mbar_init(done, 3);
+    *abort_flag = 0;
+    fence_mbar_init();
+    // pair 0: each quarter's partial rows arrive as one bulk copy of BN * 128 bytes
+    for (int q = 0; q < 4; ++q) mbar_expect_tx(&part_ready[q], BN * 128);
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, BN);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // all four CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();
+      int stage = 0;
+      uint32_t phase = 0;
+      int issues = 0;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) goto producer_done;
+        uint8_t* sa = smem + stage * S::STAGE_BYTES;
+        if (half == 0) mbar_expect_tx(&full[stage], S::TX_BYTES);
+        const uint32_t bar = mapa_shared(smem_u32(&full[stage]), lead);
+        tma_load_2d_pair(&tmA, bar, sa, kb * BK, m0);
+        tma_load_2d_pair(&tmB, bar, sa + S::A_BYTES, kb * BK, n0 + (int)half * S::BNH);
+        ++issues;
+        if (++stage == S::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    producer_done:
+      pdl_launch_dependents();
+      // the lead CTA's release commits for the stages filled last have landed here
+      if (!*abort_flag) {
+        for (int s = 0; s < S::STAGES && s < issues; ++s) {
+          int st = stage - 1 - s;
+          uint32_t ph = phase;
+          if (st < 0) {
+            st += S::STAGES;
+            ph ^= 1u;
+          }
+          mbar_wait(&empty[st], ph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+        }
+      }
+      if (*abort_flag) {  // give copies already issued time to land (their barrier is the lead CTA's)
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && half == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * BM, BN, false);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
+        const uint32_t b_addr = a_addr + S::A_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          tc_mma_f16_pair(tmem_base, sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32), idesc,
+                          (kb > kb0 || k > 0) ? 1u : 0u);
+        tc_commit_pair(&empty[stage], mask);
+        if (++stage == S::STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) tc_commit_pair(tfull, mask);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row0 = m0 + quarter * 32;
+    const int row = row0 + lane;
+    const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    pdl_wait();
+    bool ok = mbar_wait(tfull, 0, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) tc_fence_after();
+    if (split == 1) {
+      // this quarter's rows of the pair-1 accumulator, staged in this CTA's own ring (free:
+      // the pair's MMAs are done) as [BN/32 chunks][32 rows][32 columns] fp32 with the
+      // 16-byte pieces of each row swizzled by row, then one bulk copy into pair 0's ring
+      if (ok) {
+        uint8_t* mine = smem + quarter * (BN * 128);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          tmem_ld32(tb + c, v);
+          tc_wait_ld();
+          uint8_t* prow = mine + (c >> 5) * 4096 + lane * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<float4*>(prow + ((j ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        ok = __all_sync(0xffffffffu, mbar_wait_cluster(ring_free, 0, abort_flag, err, ERRBIT_TIMEOUT_GEMM));
+        if (ok && lane == 0)
+          bulk_copy_to_cluster(mapa_shared(smem_u32(mine), rank - 2), mine, BN * 128,
+                               mapa_shared(smem_u32(&part_ready[quarter]), rank - 2));
+      }
+    } else {
+      // pair 0's MMAs are done with its ring: pair 1 may fill it
+      if (ok && quarter == 0 && lane == 0) mbar_arrive_release_cluster(mapa_shared(smem_u32(ring_free), rank + 2));
+      epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0, BN);
+      if (ok) ok = __all_sync(0xffffffffu,
+                              mbar_wait_cluster(&part_ready[quarter], 0, abort_flag, err, ERRBIT_TIMEOUT_GEMM));
+      const uint8_t* part = smem + quarter * (BN * 128);
+      uint8_t* stg = smem + S::RING_BYTES + quarter * 8192;
+      uint32_t nchunk = 0;
+#pragma unroll 1
+      for (int g = 0; ok && row0 < M && g < BN; g += 128) {
+        float ssq = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          const int col = n0 + g + c;
+          float v[32];
+          tmem_ld32(tb + g + c, v);
+          tc_wait_ld();
+          const uint8_t* prow = part + ((g + c) >> 5) * 4096 + lane * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 pp = *reinterpret_cast<const float4*>(prow + ((j ^ (lane & 7)) << 4));
+            v[4 * j] += pp.x;
+            v[4 * j + 1] += pp.y;
+            v[4 * j + 2] += pp.z;
+            v[4 * j + 3] += pp.w;
+          }
+          if (row < M) {
+            epi_math<KIND, OutT>(ep, row, col, v, ssq);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          }
+          uint8_t* box = stg + (nchunk & 1) * 4096;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          stage_row(box, lane, v, (StageT*)nullptr);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (KIND == EPI_RESID)
+              tma_reduce_add_2d(&tmC, box, col, row0);
+            else
+              tma_store_2d(&tmC, box, col, row0);
+            bulk_commit();
+          }
+          ++nchunk;
+        }
+        if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
+      }
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    // every CTA of the cluster is past its last access to the others' shared memory and
+    // TMEM before any of them leaves or frees the pair's TMEM
+    if (lane == 0) {
+      for (uint32_t r = 0; r < 4; ++r)
+        if (r != rank) mbar_arrive_release_cluster(mapa_shared(smem_u32(done), r));
+      drain_wait(done, 0);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, BN);
+  }
+}
+
+template <int BN, int KIND, typename OutT>
+cudaError_t launch_tc2s(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int M, int N, int K,
+                        const EpiParams& ep, unsigned* err, cudaStream_t st) {
+  using S = Tc2Shape<BN>;
+  const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(4 * tiles);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = S::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, gemm_tc2s_kernel<BN, KIND, OutT>, a, b, c, M, N, K, ep, err);
+}
+
+template <int BN, int KIND, typename OutT>
+cudaError_t prepare_tc2s() {
+  return cudaFuncSetAttribute(gemm_tc2s_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Tc2Shape<BN>::SMEM);
+}
+
 template <int BN, int KIND, typename OutT>
 cudaError_t prepare_tc() {
   return cudaFuncSetAttribute(gemm_tc_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -572,6 +838,15 @@ cudaError_t prepare_tc() {
 }
 
 }  // namespace
+
+// clusters of four of the split-K kernel that can be resident at once, per device
+int g_split_clusters[64] = {0};
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
 
 cudaError_t gemm_tc_prepare() {
   const cudaError_t es[] = {
@@ -583,18 +858,48 @@ cudaError_t gemm_tc_prepare() {
       prepare_tc2<256, EPI_GELU, bf16>(), prepare_tc2<128, EPI_NORM, bf16>(), prepare_tc2<256, EPI_NORM, bf16>(),
       prepare_tc2<128, EPI_QKV, bf16>(), prepare_tc2<256, EPI_QKV, bf16>(), prepare_tc2<128, EPI_RESID, bf16>(),
       prepare_tc2<256, EPI_RESID, bf16>(), prepare_tc2<128, EPI_STORE, float>(),
-      prepare_tc2<256, EPI_STORE, float>()};
+      prepare_tc2<256, EPI_STORE, float>(), prepare_tc2s<256, EPI_STORE, bf16>(), prepare_tc2s<256, EPI_NORM, bf16>(),
+      prepare_tc2s<256, EPI_RESID, bf16>(), prepare_tc2s<256, EPI_STORE, float>()};
   for (cudaError_t e : es)
     if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(4 * 64);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = Tc2Shape<256>::SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_tc2s_kernel<256, EPI_RESID, bf16>, &cfg);
+  if (e != cudaSuccess) return e;
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64) g_split_clusters[dev] = n;
   return cudaSuccess;
 }
 
 cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, int M, int N, int K, int bn,
                     int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
                     bool pair) {
-  // the CTA-pair kernel stores its epilogue through the output map `c`
+  // the CTA-pair kernels store their epilogue through the output map `c`
   if (pair && !c) return cudaErrorInvalidValue;
   const CUtensorMap& cm = c ? *c : a;
+  // few 256 x 256 tiles (one per cluster of four fits the GPU): split K over two CTA pairs
+  const int tiles256 = ((M + 2 * BM - 1) / (2 * BM)) * (N / 256);
+  const int dev = current_device();
+  const int resident = dev >= 0 && dev < 64 ? g_split_clusters[dev] : 0;
+  if (pair && bn == 256 && N <= 4096 && 4 * tiles256 <= num_sms && tiles256 <= resident && K >= 2 * BK &&
+      (kind == EPI_STORE || kind == EPI_NORM || kind == EPI_RESID)) {
+    if (out_bf16) {
+      if (kind == EPI_STORE) return launch_tc2s<256, EPI_STORE, bf16>(a, b, cm, M, N, K, ep, err, st);
+      if (kind == EPI_NORM) return launch_tc2s<256, EPI_NORM, bf16>(a, b, cm, M, N, K, ep, err, st);
+      return launch_tc2s<256, EPI_RESID, bf16>(a, b, cm, M, N, K, ep, err, st);
+    }
+    if (kind == EPI_STORE) return launch_tc2s<256, EPI_STORE, float>(a, b, cm, M, N, K, ep, err, st);
+  }
 #define FH_TC_CASE(BNV, KV, OT)                                                                     \
   if (bn == BNV && kind == KV)                                                                      \
     return pair ? launch_tc2<BNV, KV, OT>(a, b, cm, M, N, K, ep, err, num_sms, st)                  \

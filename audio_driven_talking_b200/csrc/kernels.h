@@ -37,7 +37,8 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // bf16 tensor-core GEMM (gemm_tc.cu): out = epilogue(A[M,K] * W[N,K]^T); `a`, `b`
 // are TMA maps of A (box 64 x 128) and W (box 64 x bn, or 64 x bn/2 when `pair`) with
 // the 128-byte swizzle. N % bn == 0, K % 64 == 0. `pair`: 256 x bn tiles computed by
-// two CTAs of a cluster with cta_group::2; their epilogues store through `c`, a TMA map of
+// two CTAs of a cluster with cta_group::2 (bn == 256, N <= 4096 and 4 x tiles <= num_sms:
+// one tile per cluster of four, K split over two such pairs); their epilogues store through `c`, a TMA map of
 // the output (EPI_RESID: of the fp32 residual; EPI_QKV: 3D [3*B*heads][L][128]) with box
 // 32 x 32 (x 1) and the 128-byte (fp32) or 64-byte (bf16) swizzle.
 cudaError_t gemm_tc_prepare();  // sets the kernels' shared-memory attributes on the current device

@@ -26,7 +26,8 @@ def _bf16_operands(seed, M, N, K):
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (160, 256, 1536), (300, 1536, 256), (1280, 1536, 1536),
                                    (1280, 4608, 1536), (1280, 1536, 8960), (8640, 8960, 1536), (1, 128, 128),
-                                   (300, 1536, 1024), (1280, 8960, 1536)])
+                                   (300, 1536, 1024), (1280, 8960, 1536), (520, 1536, 1536), (4000, 1536, 1536),
+                                   (520, 1536, 4096), (4000, 1536, 4096)])
 def test_linear_bf16_tensor_core(M, N, K):
     """Single-CTA tiles, and 256-row CTA-pair tiles (cta_group::2) for K >= 1024, N >= 1536."""
     A, W, b = _bf16_operands(M + N + K, M, N, K)
