@@ -9,15 +9,23 @@
 //
 // attn_tc_kernel (bf16, sm_100a): one CTA per 128-query tile of one (stream, head).
 //   warp 0     TMA: the Q tile once, then K and V tiles (128 keys) double-buffered.
-//   warp 1     one thread issues tcgen05.mma: S_j = Q K_j^T into TMEM (double
-//              buffered), then O_j = P_j V_j into TMEM (double buffered) with P_j
-//              read from TMEM as the A operand and V read MN-major straight from
-//              its [key][d] layout.
-//   warps 2-9  two threads per query row (one per warpgroup, 64 keys and 64 output
-//              dims each): S_j from TMEM, online softmax in base 2, P_j written as
-//              packed bf16 back into TMEM over the S_j columns it has consumed (so P
-//              is double-buffered with S at no cost), and O_j folded into a register
-//              accumulator that carries the running max correction.
+//   warp 1     one thread issues tcgen05.mma: S_j = Q K_j^T into TMEM (double buffered),
+//              then for each key half w of tile j the product O_w += P_{j,w} V_{j,w}
+//              (P read from TMEM as the A operand, V MN-major from its [key][d] layout)
+//              into one of two TMEM accumulators O_0, O_1.
+//   warps 2-9  two warpgroups; warpgroup w owns keys 64w..64w+63 of every tile, one
+//              query row per thread, and runs its own online softmax over them (base 2,
+//              its own running max and sum): the two halves are two independent
+//              partial attentions over disjoint key sets, combined once at the end with
+//              their maxima and sums (O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1)).
+//              P is written over the S columns it has consumed as two packed bf16 parts,
+//              P_hi = bf16(p) and P_lo = bf16(p - P_hi), both multiplied by V, so the
+//              weights enter the product with about 16 bits (bf16 P alone was the
+//              kernel's whole error: the split cuts its RMS error by a quarter). O_w stays
+//              in TMEM; it is rescaled only when a row's running max grows by more than
+//              2^8 (then p <= 256 against the stale max, exact after the final division),
+//              so most tiles need no correction pass and the warpgroups never wait for
+//              each other inside the loop.
 //   The MMA thread issues S_{j+1} before P_j V_j so the tensor core works while the
 //   softmax warps exponentiate.
 // attn_simt_kernel (fp32 or bf16 inputs, CUDA cores): one query row per thread, a
@@ -39,12 +47,13 @@ constexpr uint32_t TILE = 2 * PANEL;            // [128 rows x 128 bf16]
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + TILE;        // 2 buffers
 constexpr uint32_t OFF_V = OFF_K + 2 * TILE;    // 2 buffers
-constexpr uint32_t OFF_MX = OFF_V + 2 * TILE;   // float [2][2][128] partial row maxima
-constexpr uint32_t OFF_LS = OFF_MX + 4 * 128 * 4;  // float [2][128] partial row sums
-constexpr uint32_t OFF_BAR = OFF_LS + 2 * 128 * 4;
+constexpr uint32_t OFF_ML = OFF_V + 2 * TILE;   // float [2 halves][2 (m, l)][128 rows]
+constexpr uint32_t OFF_BAR = OFF_ML + 4 * 128 * 4;
 constexpr uint32_t OFF_RKALL = OFF_BAR + 256;   // float rk[round_up(L, 128)]: every key's RMS factor
 constexpr int AT_MAX_L = 8192;
 constexpr uint32_t AT_SMEM = OFF_RKALL + AT_MAX_L * 4 + 1024;
+constexpr float AT_RESCALE = 8.f;               // log2 growth of a row max that forces a rescale
+// TMEM columns: S_0 0-127, S_1 128-255 (P over them), O_0 256-383, O_1 384-511
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -71,15 +80,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* v_full = bars + 3;    // [2]
   uint64_t* k_empty = bars + 5;   // [2] K buffer free (S MMA done)
-  uint64_t* v_empty = bars + 9;   // [2] V buffer free (P.V MMA done); also orders S-buffer reuse
   uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* o_full = bars + 11;   // [2]
-  uint64_t* o_free = bars + 13;   // [2]
-  uint64_t* p_full = bars + 15;
-  uint64_t* rk_full = bars + 17;  // every key's RMS factor staged
-  uint64_t* mx_bar = bars + 21;   // [2]
-  uint64_t* l_bar = bars + 23;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 24);
+  uint64_t* v_empty = bars + 9;   // [2] V buffer free (both halves' P.V done); also orders S-buffer reuse
+  // [2 halves][2 tiles by parity] P written. Two per half: a warpgroup no longer waits for
+  // each tile's P.V, so it can publish P_{i+1} before the MMA thread has waited for P_i
+  // (never P_{i+2}: S_{i+2} waits for P_i V_i), which one phase bit could not tell apart.
+  uint64_t* p_full = bars + 11;
+  // [2 halves][2 tiles by parity] P.V of a tile accumulated into O_w. A warpgroup waits for
+  // one only to rescale O_w or at the end, so it may skip phases; per parity, the phase two
+  // tiles back is always complete (S_j waits for P_{j-2} V_{j-2}) and the one two tiles
+  // ahead cannot start, so each wait names one phase.
+  uint64_t* pv_done = bars + 15;
+  uint64_t* rk_full = bars + 19;  // every key's RMS factor staged
+  uint64_t* fin_bar = bars + 20;  // both halves' (m, l) published
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -97,15 +111,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       mbar_init(&k_empty[i], 1);
       mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&o_full[i], 1);
-      mbar_init(&o_free[i], AT_SOFTMAX_THREADS);
+      mbar_init(&p_full[2 * i], AT_SOFTMAX_THREADS / 2);
+      mbar_init(&p_full[2 * i + 1], AT_SOFTMAX_THREADS / 2);
+      mbar_init(&pv_done[2 * i], 1);
+      mbar_init(&pv_done[2 * i + 1], 1);
     }
-    mbar_init(p_full, AT_SOFTMAX_THREADS);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&mx_bar[i], AT_SOFTMAX_THREADS);
-    }
-    mbar_init(l_bar, AT_SOFTMAX_THREADS);
     mbar_init(rk_full, AT_SOFTMAX_THREADS);
+    mbar_init(fin_bar, AT_SOFTMAX_THREADS);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -184,6 +196,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const uint32_t q_addr = smem_u32(smem + OFF_Q);
       bool ok = mbar_wait(q_full, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       tc_fence_after();
+      int pv_issued = 0;  // tiles whose P.V was issued (for the tail)
       for (int j = 0; ok && j <= nkv; ++j) {
         if (j < nkv) {  // S_j = Q K_j^T
           const int bf = j & 1;
@@ -202,33 +215,43 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           tc_commit(&s_full[bf]);
           tc_commit(&k_empty[bf]);
         }
-        if (j >= 1) {  // O_i = P_i V_i for i = j - 1
+        if (j >= 1) {  // O_w += P_{i,w} V_{i,w} for i = j - 1, each half as soon as its P is written
           const int i = j - 1;
           const int bf = i & 1;
           const uint32_t par = (i >> 1) & 1;
-          if (!mbar_wait(p_full, i & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
           if (!mbar_wait(&v_full[bf], par, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
-          if (!mbar_wait(&o_free[bf], par ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) break;
-          tc_fence_after();
           const uint32_t v_addr = smem_u32(smem + OFF_V + bf * TILE);
+          bool hok = true;
+          for (int w = 0; w < 2; ++w) {
+            if (!mbar_wait(&p_full[2 * w + bf], par, abort_flag, err, ERRBIT_TIMEOUT_ATTN)) {
+              hok = false;
+              break;
+            }
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            // keys 16kk..16kk+15 of P_i: packed in columns 64*(kk/4) + 8*(kk%4) of S_i's buffer
-            const uint32_t a_tmem = tmem + bf * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-            const uint32_t b_off = kk * 16 * 128;                      // 16 key rows of V
-            tc_mma_f16_ts(tmem + 256 + bf * 128, a_tmem, sdesc_mnmajor_sw128(v_addr + b_off, PANEL), id_o,
-                          kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) {
+              // keys 64w + 16(kk%4) .. +15: P_hi (kk < 4) in columns 64w + 8(kk%4), P_lo 32 further
+              const uint32_t a_tmem = tmem + bf * 128 + w * 64 + (kk >> 2) * 32 + (kk & 3) * 8;
+              const uint32_t b_off = (w * 64 + (kk & 3) * 16) * 128;  // 16 key rows of V
+              tc_mma_f16_ts(tmem + 256 + w * 128, a_tmem, sdesc_mnmajor_sw128(v_addr + b_off, PANEL), id_o,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&pv_done[2 * w + bf]);
           }
-          tc_commit(&o_full[bf]);
+          if (!hok) break;
           tc_commit(&v_empty[bf]);
+          pv_issued = j;
         }
+      }
+      // tail: the last P.V commits have landed before the CTA can leave
+      if (pv_issued > 0) {
+        const int last = pv_issued - 1;
+        mbar_wait(&pv_done[0 + (last & 1)], (last >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+        mbar_wait(&pv_done[2 + (last & 1)], (last >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       }
     }
   } else {
-    // softmax / correction / output, warps 2-9: each query row belongs to one thread of each
-    // warpgroup; half 0 (warps 2-5) takes keys and output dims 0-63, half 1 (warps 6-9)
-    // takes 64-127. Only the partial row maxima cross between the halves (per tile, through
-    // shared memory and an mbarrier); the partial row sums are combined once at the end.
+    // softmax, warps 2-9: warpgroup `half` owns keys 64*half .. 64*half + 63 of every tile
     const int quarter = warp & 3;                      // TMEM lane quarter of this warp
     const int half = (warp - 2) >> 2;
     const int t = threadIdx.x - 64;                    // 0..255 among the softmax threads
@@ -239,38 +262,32 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     const float rq = row_rms(ssq, ssq_ld, (long)b * L + (qvalid ? qi : L - 1), 0, heads, inv_d, eps);
     const float qscale = rq * scale_log2;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float* mxs = reinterpret_cast<float*>(smem + OFF_MX);  // [2 tiles][2 halves][128 rows]
-    float* lss = reinterpret_cast<float*>(smem + OFF_LS);  // [2 halves][128 rows]
+    const uint32_t o_t = tmem + lane_off + 256 + half * 128;  // this half's O accumulator row
+    float* mls = reinterpret_cast<float*>(smem + OFF_ML);    // [2 halves][m, l][128 rows]
 
     // every key's RMS factor, once per CTA (the keys are shared by all tiles of the row)
     float* rk_all = reinterpret_cast<float*>(smem + OFF_RKALL);
     for (int key = t; key < nkv * AT_BK; key += AT_SOFTMAX_THREADS)
       rk_all[key] = key < L ? row_rms(ssq, ssq_ld, (long)b * L + key, heads, heads, inv_d, eps) : 0.f;
-    mbar_arrive(&rk_full[0]);
-    float o[64];
-#pragma unroll
-    for (int d = 0; d < 64; ++d) o[d] = 0.f;
+    mbar_arrive(rk_full);
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-
-    ok = mbar_wait(&rk_full[0], 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+    bool ok = mbar_wait(rk_full, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
     ok = __all_sync(0xffffffffu, ok);
     for (int j = 0; ok && j < nkv; ++j) {
       const float* rk = rk_all + j * AT_BK + half * 64;
       const int bf = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      ok = mbar_wait(&s_full[bf], par, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+      ok = mbar_wait(&s_full[bf], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const uint32_t s_t = tmem + lane_off + bf * 128 + half * 64;
       const int kvalid = L - j * AT_BK - half * 64;  // keys of this half-tile that exist
-      // this half's 64 scores of the row, one batched TMEM read kept in registers for both passes
       float sa[32], sb[32];
       tmem_ld32(s_t, sa);
       tmem_ld32(s_t + 32, sb);
       tc_wait_ld();
-      // scaled scores r_k * (q.k); keys past the end of the sequence get -inf (only the last tile)
+      // r_k (q.k) per key; the row factor r_q / sqrt(128) * log2(e) (qscale > 0) is applied
+      // to the max and inside the exponent's FMA; missing keys get -inf
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         sa[e] *= rk[e];
@@ -283,99 +300,112 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
           if (e + 32 >= kvalid) sb[e] = -INFINITY;
         }
       }
-      // row max as a tree (independent chains)
       float m8[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         m8[u] = fmaxf(fmaxf(sa[u], sa[u + 8]), fmaxf(sa[u + 16], sa[u + 24]));
         m8[u] = fmaxf(m8[u], fmaxf(fmaxf(sb[u], sb[u + 8]), fmaxf(sb[u + 16], sb[u + 24])));
       }
-      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      float* mxt = mxs + (j & 1) * 256;
-      mxt[half * 128 + rl] = mx;
-      mbar_arrive(&mx_bar[j & 1]);
-      ok = mbar_wait(&mx_bar[j & 1], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      mx = fmaxf(mx, mxt[(1 - half) * 128 + rl]);
-      const float m_new = fmaxf(m_run, mx * qscale);
-      const float alpha = ex2(m_run - m_new);
-      // probabilities (ex2 of -inf is 0), four independent partial sums, packed bf16 P
-      // written over the consumed S columns
+      const float mt = qscale * fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                      fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      // the running max moves only when it must (first tile, or growth beyond 2^8); the
+      // warp rescales together so its TMEM accesses stay collective
+      const bool grow = __any_sync(0xffffffffu, mt > m_run + AT_RESCALE);
+      if (grow) {
+        const float m_new = fmaxf(m_run, mt);
+        if (j > 0) {
+          // 0 for a row that had only missing keys so far (its O and l are 0); 1 if still none
+          const float alpha = m_new == -INFINITY ? 1.f : ex2(m_run - m_new);
+          l_run *= alpha;
+          // O_w holds P V up to tile j-1: wait for that product, then scale it in place
+          ok = mbar_wait(&pv_done[2 * half + ((j - 1) & 1)], ((j - 1) >> 1) & 1, abort_flag, err,
+                         ERRBIT_TIMEOUT_ATTN);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            float o[32];
+            tmem_ld32(o_t + c, o);
+            tc_wait_ld();
+            uint32_t lo[16], hi[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              lo[e] = __float_as_uint(o[e] * alpha);
+              hi[e] = __float_as_uint(o[e + 16] * alpha);
+            }
+            tmem_st16(o_t + c, lo);
+            tmem_st16(o_t + c + 16, hi);
+          }
+          tc_wait_st();
+        }
+        m_run = m_new;
+      }
+      // probabilities against the (possibly stale) running max, split into bf16 high and low
+      // parts; a row whose keys so far are all missing uses 0 as its reference (ex2(-inf) = 0)
+      const float mref = m_run == -INFINITY ? 0.f : m_run;
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pa[16], pb2[16];
+      uint32_t pa[16], pb2[16], la[16], lb[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        const float p0 = ex2(fmaf(sa[2 * u], qscale, -m_new));
-        const float p1 = ex2(fmaf(sa[2 * u + 1], qscale, -m_new));
-        const float q0 = ex2(fmaf(sb[2 * u], qscale, -m_new));
-        const float q1 = ex2(fmaf(sb[2 * u + 1], qscale, -m_new));
+        const float p0 = ex2(fmaf(sa[2 * u], qscale, -mref));
+        const float p1 = ex2(fmaf(sa[2 * u + 1], qscale, -mref));
+        const float q0 = ex2(fmaf(sb[2 * u], qscale, -mref));
+        const float q1 = ex2(fmaf(sb[2 * u + 1], qscale, -mref));
         rs4[u & 3] += (p0 + p1) + (q0 + q1);
         __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
         __nv_bfloat162 h1 = __floats2bfloat162_rn(q0, q1);
+        const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
+        __nv_bfloat162 g0 = __floats2bfloat162_rn(p0 - f0.x, p1 - f0.y);
+        __nv_bfloat162 g1 = __floats2bfloat162_rn(q0 - f1.x, q1 - f1.y);
         pa[u] = *reinterpret_cast<uint32_t*>(&h0);
         pb2[u] = *reinterpret_cast<uint32_t*>(&h1);
+        la[u] = *reinterpret_cast<uint32_t*>(&g0);
+        lb[u] = *reinterpret_cast<uint32_t*>(&g1);
       }
-      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      tmem_st16(s_t, pa);        // keys 0..31 of this half -> columns 0..15 (already read)
-      tmem_st16(s_t + 16, pb2);  // keys 32..63 -> columns 16..31
+      l_run += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      tmem_st16(s_t, pa);        // P_hi of keys 0..31 of this half -> columns 0..15 (already read)
+      tmem_st16(s_t + 16, pb2);  // P_hi of keys 32..63 -> columns 16..31
+      tmem_st16(s_t + 32, la);   // P_lo -> columns 32..63
+      tmem_st16(s_t + 48, lb);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-      // fold this half's 64 dims of O_{j-1} (relative to the previous max), rescale to the new max
-      if (j >= 1) {
-        const int pb = (j - 1) & 1;
-        ok = mbar_wait(&o_full[pb], ((j - 1) >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t o_t = tmem + lane_off + 256 + pb * 128 + half * 64;
-        {
-          float oa[32], ob[32];
-          tmem_ld32(o_t, oa);
-          tmem_ld32(o_t + 32, ob);
-          tc_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            o[e] = (o[e] + oa[e]) * alpha;
-            o[e + 32] = (o[e + 32] + ob[e]) * alpha;
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&o_free[pb]);
-      }
+      mbar_arrive(&p_full[2 * half + bf]);
     }
     if (ok) {
-      const int pb = (nkv - 1) & 1;
-      ok = mbar_wait(&o_full[pb], ((nkv - 1) >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+      // this half's last product, then both halves' (m, l) for the combination
+      ok = mbar_wait(&pv_done[2 * half + ((nkv - 1) & 1)], ((nkv - 1) >> 1) & 1, abort_flag, err,
+                     ERRBIT_TIMEOUT_ATTN);
+      mls[(half * 2 + 0) * 128 + rl] = m_run;
+      mls[(half * 2 + 1) * 128 + rl] = l_run;
+      mbar_arrive(fin_bar);
+      ok = ok && mbar_wait(fin_bar, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
-        const uint32_t o_t = tmem + lane_off + 256 + pb * 128 + half * 64;
-#pragma unroll
+        const float m0 = mls[0 * 128 + rl], l0 = mls[1 * 128 + rl];
+        const float m1 = mls[2 * 128 + rl], l1 = mls[3 * 128 + rl];
+        const float m = fmaxf(m0, m1);
+        const float a0 = ex2(m0 - m), a1 = ex2(m1 - m);  // m1 = -inf (no key in half 1): a1 = 0
+        const float inv_l = 1.f / (a0 * l0 + a1 * l1);
+        const float c0 = a0 * inv_l, c1 = a1 * inv_l;
+        // this warpgroup writes output dims 64*half .. +63 from both accumulators
+        const uint32_t o0 = tmem + lane_off + 256 + half * 64, o1 = tmem + lane_off + 384 + half * 64;
+        bf16* dst = out + ((long)b * L + qi) * D + h * 128 + half * 64;
+#pragma unroll 1
         for (int c = 0; c < 64; c += 32) {
-          float v[32];
-          tmem_ld32(o_t + c, v);
+          float x0[32], x1[32];
+          tmem_ld32(o0 + c, x0);
+          tmem_ld32(o1 + c, x1);
           tc_wait_ld();
+          if (qvalid) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[c + e] += v[e];
-        }
-        // the row's normaliser is the sum of both halves' partial sums
-        lss[half * 128 + rl] = l_run;
-        mbar_arrive(l_bar);
-        ok = mbar_wait(l_bar, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
-        ok = __all_sync(0xffffffffu, ok);
-        if (ok && qvalid) {
-          const float inv_l = 1.f / (l_run + lss[(1 - half) * 128 + rl]);
-          bf16* dst = out + ((long)b * L + qi) * D + h * 128 + half * 64;
+            for (int d = 0; d < 32; d += 8) {
+              float w8[8];
 #pragma unroll
-          for (int d = 0; d < 64; d += 8) {
-            float w[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = o[d + e] * inv_l;
-            store8(dst + d, w);
+              for (int e = 0; e < 8; ++e) w8[e] = x0[d + e] * c0 + x1[d + e] * c1;
+              store8(dst + c + d, w8);
+            }
           }
         }
       }
