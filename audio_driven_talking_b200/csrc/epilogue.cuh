@@ -127,6 +127,10 @@ __device__ __forceinline__ void epi_prefetch(const EpiParams& p, int row, int co
       if (epi_normed(p, col0 + c)) prefetch_l1(p.gain + col0 + c);
     }
   }
+  if constexpr (KIND == EPI_QKV) {  // the row's rotary angles (64 (cos, sin) pairs, 4 lines)
+    const float2* rt = p.rope + (long)(row % p.rows_per_batch) * 64;
+    for (int c = 0; c < 64; c += 16) prefetch_l1(rt + c);
+  }
 }
 
 // epi_math plus the store by the owning thread (row-major outputs, the residual update,

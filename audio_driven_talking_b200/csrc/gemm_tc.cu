@@ -338,20 +338,35 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      // The weights W are never written by any kernel: stream the first stages' W halves
+      // before waiting for the kernels this one depends on (programmatic launch).
+      int pre = 0;
+      if (cl < ntiles) {
+        const int n0 = (cl / num_m) * BN + (int)rank * S::BNH;
+        pre = nk < S::STAGES ? nk : S::STAGES;
+        for (int s = 0; s < pre; ++s) {
+          if (rank == 0) mbar_expect_tx(&full[s], S::TX_BYTES);
+          tma_load_2d_pair(&tmB, mapa_shared(smem_u32(&full[s]), 0), smem + s * S::STAGE_BYTES + S::A_BYTES, s * BK,
+                           n0);
+        }
+      }
       pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
       int issues = 0;
-      for (int tile = cl; tile < ntiles; tile += ncl) {
+      bool first = true;
+      for (int tile = cl; tile < ntiles; tile += ncl, first = false) {
         const int m0 = (tile % num_m) * 2 * BM + (int)rank * BM;
         const int n0 = (tile / num_m) * BN + (int)rank * S::BNH;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) goto producer_done;
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
-          if (rank == 0) mbar_expect_tx(&full[stage], S::TX_BYTES);
           const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+          if (!(first && kb < pre)) {
+            if (rank == 0) mbar_expect_tx(&full[stage], S::TX_BYTES);
+            tma_load_2d_pair(&tmB, bar0, sa + S::A_BYTES, kb * BK, n0);
+          }
           tma_load_2d_pair(&tmA, bar0, sa, kb * BK, m0);
-          tma_load_2d_pair(&tmB, bar0, sa + S::A_BYTES, kb * BK, n0);
           ++issues;
           if (++stage == S::STAGES) {
             stage = 0;
@@ -636,6 +651,13 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
+      // the first stages' W halves before the dependency wait (W is never written)
+      const int pre = kb1 - kb0 < S::STAGES ? kb1 - kb0 : S::STAGES;
+      for (int s = 0; s < pre; ++s) {
+        if (half == 0) mbar_expect_tx(&full[s], S::TX_BYTES);
+        tma_load_2d_pair(&tmB, mapa_shared(smem_u32(&full[s]), lead), smem + s * S::STAGE_BYTES + S::A_BYTES,
+                         (kb0 + s) * BK, n0 + (int)half * S::BNH);
+      }
       pdl_wait();
       int stage = 0;
       uint32_t phase = 0;
@@ -643,10 +665,12 @@ __global__ void __launch_bounds__(192, 1)
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) goto producer_done;
         uint8_t* sa = smem + stage * S::STAGE_BYTES;
-        if (half == 0) mbar_expect_tx(&full[stage], S::TX_BYTES);
         const uint32_t bar = mapa_shared(smem_u32(&full[stage]), lead);
+        if (kb - kb0 >= pre) {
+          if (half == 0) mbar_expect_tx(&full[stage], S::TX_BYTES);
+          tma_load_2d_pair(&tmB, bar, sa + S::A_BYTES, kb * BK, n0 + (int)half * S::BNH);
+        }
         tma_load_2d_pair(&tmA, bar, sa, kb * BK, m0);
-        tma_load_2d_pair(&tmB, bar, sa + S::A_BYTES, kb * BK, n0 + (int)half * S::BNH);
         ++issues;
         if (++stage == S::STAGES) {
           stage = 0;
