@@ -54,7 +54,8 @@ def slice_tflop() -> float:
 
 
 # launches per class inside one slice, and each launch's algorithmic flops
-CLASS_NAMES = {1: "gemm_tc2_kernel<128,EPI_RESID> (CTA pair; O-proj, cross-O, FFN2 with gated residual)",
+CLASS_NAMES = {1: "gated-residual GEMMs: gemm_tc2_kernel<128,EPI_RESID> (CTA pair; O-proj, cross-O) and "
+                  "gemm_tc2s_kernel<256,EPI_RESID> (split-K on clusters of four; FFN2)",
                2: "gemm_tc2_kernel<256,EPI_GELU> (CTA pair; FFN1)"}
 
 
