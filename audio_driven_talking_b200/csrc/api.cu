@@ -123,8 +123,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // QKV, O-proj, cross-Q/O, FFN1, FFN2) run as 256-row tiles on CTA pairs (cta_group::2),
 // each CTA streaming half of the W tile; the rest (patch embed K=256, head N=128, the
 // per-slice cross-KV with 160 rows) on single CTAs. Tile width 256 for FFN1, the cross-KV
-// and FFN2 (split-K on clusters of four at 1280 tokens); 128 for QKV and the K = 1536
-// projections (measured on B200 at 1280 tokens).
+// and the width-1536 projections (split-K on clusters of four at 1280 tokens); 128 for QKV
+// (measured on B200 at 1280 tokens).
 struct TileCfg {
   int bn;
   bool pair;
@@ -133,11 +133,10 @@ struct TileCfg {
 TileCfg tile_cfg(int N, int K, bool pair_ok = true) {
   TileCfg t;
   t.pair = pair_ok && K >= 1024 && N >= 1536 && N <= 16384;
-  // 256 wide for FFN1 and the cross-KV, and for deep-K pair GEMMs of width up to 4096
-  // (FFN2), which then run split-K on clusters of four when their 256 x 256 tiles are few
-  // (kernels.h); the K = 1536 projections of width 1536 stay at 128 (their main loop is too
-  // short to repay the split's reduction)
-  t.bn = (N % 256 == 0 && (N >= 8192 || (t.pair && N <= 4096 && K >= 4096))) ? 256 : 128;
+  // 256 wide for FFN1 and the cross-KV, and for the pair GEMMs of width up to 4096 (O-proj,
+  // cross-Q/O, FFN2), which then run split-K on clusters of four when their 256 x 256 tiles
+  // are few (kernels.h); 128 for QKV
+  t.bn = (N % 256 == 0 && (N >= 8192 || (t.pair && N <= 4096))) ? 256 : 128;
   t.wbox = t.pair ? t.bn / 2 : t.bn;
   return t;
 }

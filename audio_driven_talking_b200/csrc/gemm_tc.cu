@@ -585,26 +585,31 @@ cudaError_t prepare_tc2() {
 // GEMMs with few output tiles (M = 1280, N = 1536: 30 tiles of 256 x 256) run one tile per
 // cluster of four CTAs. CTA pair s (cluster ranks 2s, 2s+1) computes the tile over half of
 // the K range with cta_group::2 MMAs into its own TMEM accumulator, on 256-wide tiles whose
-// operand traffic per MMA is the lowest the pair can have. Pair 1's epilogue warps then
-// write their fp32 accumulator rows into pair 0's shared memory (the operand ring, free
-// once pair 0's MMAs are done) and pair 0 adds them to its own, always in that order,
-// before the usual staged epilogue. One tile per cluster: the host launches this only
-// when 4 x tiles CTAs fit on the GPU.
+// operand traffic per MMA is the lowest the pair can have. The pairs then reduce-scatter
+// through shared memory: each CTA finalises 128 of the 256 columns of its rows, receiving
+// the partner pair's fp32 partial sums for them by one bulk copy per warp into its operand
+// ring (free once its pair's MMAs are done), adding them to its own and running the staged
+// epilogue. One tile per cluster: the host launches this only when the tiles fit the
+// clusters of four that can be resident at once.
 template <int BN, int KIND, typename OutT>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc2s_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep, unsigned* err) {
   using S = Tc2Shape<BN>;
   static_assert(KIND != EPI_QKV, "the head-major scatter runs on the plain pair kernel");
-  static_assert(BN * 512 <= (int)S::RING_BYTES, "the partial accumulator must fit in the operand ring");
+  static_assert(BN == 256, "each CTA finalises one 128-column group");
+  constexpr uint32_t HALF_COLS = BN / 2;
+  constexpr uint32_t QBYTES = HALF_COLS * 128;   // one quarter's rows of half the columns, fp32
+  constexpr uint32_t RX = 4 * QBYTES;            // ring offset of the partner's half
+  static_assert(2 * RX <= S::RING_BYTES, "both halves must fit in the operand ring");
   using StageT = typename std::conditional<KIND == EPI_RESID, float, OutT>::type;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::RING_BYTES + S::STG_BYTES);
   uint64_t* empty = full + S::STAGES;
   uint64_t* tfull = empty + S::STAGES;
-  uint64_t* ring_free = tfull + 1;   // on pair 1: pair 0's ring may be overwritten
-  uint64_t* part_ready = ring_free + 1;  // [4] on pair 0: a quarter's partial rows have landed
+  uint64_t* ring_free = tfull + 1;       // the partner's MMAs are done: its ring may be written
+  uint64_t* part_ready = ring_free + 1;  // [4] the partner's half of a quarter's rows has landed
   uint64_t* done = part_ready + 4;   // every other CTA of the cluster is finished with this one
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -634,8 +639,8 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(done, 3);
     *abort_flag = 0;
     fence_mbar_init();
-    // pair 0: each quarter's partial rows arrive as one bulk copy of BN * 128 bytes
-    for (int q = 0; q < 4; ++q) mbar_expect_tx(&part_ready[q], BN * 128);
+    // each quarter's rows of the columns this CTA finalises arrive as one bulk copy
+    for (int q = 0; q < 4; ++q) mbar_expect_tx(&part_ready[q], QBYTES);
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmC);
@@ -732,83 +737,84 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = mbar_wait(tfull, 0, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) tc_fence_after();
-    if (split == 1) {
-      // this quarter's rows of the pair-1 accumulator, staged in this CTA's own ring (free:
-      // the pair's MMAs are done) as [BN/32 chunks][32 rows][32 columns] fp32 with the
-      // 16-byte pieces of each row swizzled by row, then one bulk copy into pair 0's ring
-      if (ok) {
-        uint8_t* mine = smem + quarter * (BN * 128);
+    // Reduce-scatter between the pairs: the CTA finalises columns [mine, mine + BN/2) of its
+    // 128 rows and its partner (same rows, other half of K, cluster rank ^ 2) the other
+    // half. Each stages the partner's half of its accumulator in its own ring (free: its
+    // pair's MMAs are done) as [BN/64 chunks][32 rows][32 columns] fp32 per quarter with
+    // the 16-byte pieces of each row swizzled by row, and one bulk copy per warp moves it
+    // into the partner's ring at offset RX once the partner's MMAs are done with it.
+    const uint32_t partner = rank ^ 2u;
+    const int mine = (int)split * (int)HALF_COLS, theirs = (int)HALF_COLS - mine;
+    if (ok && quarter == 0 && lane == 0) mbar_arrive_release_cluster(mapa_shared(smem_u32(ring_free), partner));
+    epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0 + mine, HALF_COLS);
+    if (ok && row0 < M) {
+      uint8_t* out = smem + quarter * QBYTES;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          float v[32];
-          tmem_ld32(tb + c, v);
-          tc_wait_ld();
-          uint8_t* prow = mine + (c >> 5) * 4096 + lane * 128;
+      for (int c = 0; c < (int)HALF_COLS; c += 32) {
+        float v[32];
+        tmem_ld32(tb + theirs + c, v);
+        tc_wait_ld();
+        uint8_t* prow = out + (c >> 5) * 4096 + lane * 128;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<float4*>(prow + ((j ^ (lane & 7)) << 4)) =
-                make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        ok = __all_sync(0xffffffffu, mbar_wait_cluster(ring_free, 0, abort_flag, err, ERRBIT_TIMEOUT_GEMM));
-        if (ok && lane == 0)
-          bulk_copy_to_cluster(mapa_shared(smem_u32(mine), rank - 2), mine, BN * 128,
-                               mapa_shared(smem_u32(&part_ready[quarter]), rank - 2));
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(prow + ((j ^ (lane & 7)) << 4)) =
+              make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
       }
-    } else {
-      // pair 0's MMAs are done with its ring: pair 1 may fill it
-      if (ok && quarter == 0 && lane == 0) mbar_arrive_release_cluster(mapa_shared(smem_u32(ring_free), rank + 2));
-      epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0, BN);
+      fence_proxy_async_smem();
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, mbar_wait_cluster(ring_free, 0, abort_flag, err, ERRBIT_TIMEOUT_GEMM));
+      if (ok && lane == 0)
+        bulk_copy_to_cluster(mapa_shared(smem_u32(smem + RX + quarter * QBYTES), partner), out, QBYTES,
+                             mapa_shared(smem_u32(&part_ready[quarter]), partner));
       if (ok) ok = __all_sync(0xffffffffu,
                               mbar_wait_cluster(&part_ready[quarter], 0, abort_flag, err, ERRBIT_TIMEOUT_GEMM));
-      const uint8_t* part = smem + quarter * (BN * 128);
-      uint8_t* stg = smem + S::RING_BYTES + quarter * 8192;
-      uint32_t nchunk = 0;
-#pragma unroll 1
-      for (int g = 0; ok && row0 < M && g < BN; g += 128) {
-        float ssq = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          const int col = n0 + g + c;
-          float v[32];
-          tmem_ld32(tb + g + c, v);
-          tc_wait_ld();
-          const uint8_t* prow = part + ((g + c) >> 5) * 4096 + lane * 128;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 pp = *reinterpret_cast<const float4*>(prow + ((j ^ (lane & 7)) << 4));
-            v[4 * j] += pp.x;
-            v[4 * j + 1] += pp.y;
-            v[4 * j + 2] += pp.z;
-            v[4 * j + 3] += pp.w;
-          }
-          if (row < M) {
-            epi_math<KIND, OutT>(ep, row, col, v, ssq);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = 0.f;
-          }
-          uint8_t* box = stg + (nchunk & 1) * 4096;
-          if (lane == 0) bulk_wait_read<1>();
-          __syncwarp();
-          stage_row(box, lane, v, (StageT*)nullptr);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if constexpr (KIND == EPI_RESID)
-              tma_reduce_add_2d(&tmC, box, col, row0);
-            else
-              tma_store_2d(&tmC, box, col, row0);
-            bulk_commit();
-          }
-          ++nchunk;
-        }
-        if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
-      }
-      if (lane == 0) bulk_wait_all();
-      __syncwarp();
     }
+    // the finalised half: own accumulator + the partner's, then the staged epilogue
+    const uint8_t* part = smem + RX + quarter * QBYTES;
+    uint8_t* stg = smem + S::RING_BYTES + quarter * 8192;
+    uint32_t nchunk = 0;
+    if (ok && row0 < M) {
+      float ssq = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < (int)HALF_COLS; c += 32) {
+        const int col = n0 + mine + c;
+        float v[32];
+        tmem_ld32(tb + mine + c, v);
+        tc_wait_ld();
+        const uint8_t* prow = part + (c >> 5) * 4096 + lane * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 pp = *reinterpret_cast<const float4*>(prow + ((j ^ (lane & 7)) << 4));
+          v[4 * j] += pp.x;
+          v[4 * j + 1] += pp.y;
+          v[4 * j + 2] += pp.z;
+          v[4 * j + 3] += pp.w;
+        }
+        if (row < M) {
+          epi_math<KIND, OutT>(ep, row, col, v, ssq);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.f;
+        }
+        uint8_t* box = stg + (nchunk & 1) * 4096;
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        stage_row(box, lane, v, (StageT*)nullptr);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (KIND == EPI_RESID)
+            tma_reduce_add_2d(&tmC, box, col, row0);
+          else
+            tma_store_2d(&tmC, box, col, row0);
+          bulk_commit();
+        }
+        ++nchunk;
+      }
+      if (row < M) epi_group_end<KIND>(ep, row, n0 + mine, ssq);
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
