@@ -122,9 +122,9 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Tile shape per GEMM, from the weight's N and K. Deep projections (K >= 1024, N >= 1536:
 // QKV, O-proj, cross-Q/O, FFN1, FFN2) run as 256-row tiles on CTA pairs (cta_group::2),
 // each CTA streaming half of the W tile; the rest (patch embed K=256, head N=128, the
-// per-slice cross-KV with 160 rows) on single CTAs. Tile width 256 for FFN1, the cross-KV
-// and the width-1536 projections (split-K on clusters of four at 1280 tokens); 128 for QKV
-// (measured on B200 at 1280 tokens).
+// per-slice cross-KV with 160 rows) on single CTAs. Tile width 224 for FFN1, 256 for the
+// cross-KV and the width-1536 projections (split-K on clusters of four at 1280 tokens), 128
+// for QKV (measured on B200 at 1280 tokens).
 struct TileCfg {
   int bn;
   bool pair;
@@ -137,6 +137,9 @@ TileCfg tile_cfg(int N, int K, bool pair_ok = true) {
   // cross-Q/O, FFN2), which then run split-K on clusters of four when their 256 x 256 tiles
   // are few (kernels.h); 128 for QKV
   t.bn = (N % 256 == 0 && (N >= 8192 || (t.pair && N <= 4096))) ? 256 : 128;
+  // FFN1 (N = 8960 = 40 x 224): at 1280 tokens 200 pair tiles of width 224 fill three rounds
+  // of 74 CTA pairs better than 175 tiles of width 256
+  if (t.pair && N >= 8192 && N % 224 == 0) t.bn = 224;
   t.wbox = t.pair ? t.bn / 2 : t.bn;
   return t;
 }

@@ -271,7 +271,9 @@ cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, 
 template <int BN>
 struct Tc2Shape {
   static constexpr int BNH = BN / 2;
-  static constexpr int STAGES = (BN == 256) ? 6 : 8;
+  static constexpr int STAGES = (BN >= 192) ? 6 : 8;
+  // two accumulators of BN columns, allocated as a power of two
+  static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
   static constexpr uint32_t A_BYTES = BM * BK * 2;
   static constexpr uint32_t B_BYTES = BNH * BK * 2;
   static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -328,7 +330,7 @@ __global__ void __launch_bounds__(192, 1)
     if (STAGED) prefetch_tmap(&tmC);
   }
   if (warp == 1) {
-    tmem_alloc_pair(tmem_holder, 2 * BN);
+    tmem_alloc_pair(tmem_holder, S::TMEM_COLS);
     tmem_relinquish_pair();
   }
   tc_fence_before();
@@ -471,7 +473,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int g = 0; row0 < M && g < BN; g += 128) {  // a warp with no row below M stores nothing
           float ssq = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
+          for (int c = 0; c < 128 && g + c < BN; c += 32) {
             float v[32];
             tmem_ld32(tb + g + c, v);
             tc_wait_ld();
@@ -521,7 +523,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int g = 0; g < BN; g += 128) {
           float ssq = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
+          for (int c = 0; c < 128 && g + c < BN; c += 32) {
             float v[32];
             tmem_ld32(tb + g + c, v);
             tc_wait_ld();
@@ -547,7 +549,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, 2 * BN);
+    tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
   }
 }
 
@@ -888,7 +890,7 @@ cudaError_t gemm_tc_prepare() {
       prepare_tc2<256, EPI_GELU, bf16>(), prepare_tc2<128, EPI_NORM, bf16>(), prepare_tc2<256, EPI_NORM, bf16>(),
       prepare_tc2<128, EPI_QKV, bf16>(), prepare_tc2<256, EPI_QKV, bf16>(), prepare_tc2<128, EPI_RESID, bf16>(),
       prepare_tc2<256, EPI_RESID, bf16>(), prepare_tc2<128, EPI_STORE, float>(),
-      prepare_tc2<256, EPI_STORE, float>(), prepare_tc2s<256, EPI_STORE, bf16>(), prepare_tc2s<256, EPI_NORM, bf16>(),
+      prepare_tc2<256, EPI_STORE, float>(), prepare_tc2<224, EPI_GELU, bf16>(), prepare_tc2<224, EPI_STORE, float>(), prepare_tc2s<256, EPI_STORE, bf16>(), prepare_tc2s<256, EPI_NORM, bf16>(),
       prepare_tc2s<256, EPI_RESID, bf16>(), prepare_tc2s<256, EPI_STORE, float>()};
   for (cudaError_t e : es)
     if (e != cudaSuccess) return e;
@@ -934,6 +936,12 @@ cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
   if (bn == BNV && kind == KV)                                                                      \
     return pair ? launch_tc2<BNV, KV, OT>(a, b, cm, M, N, K, ep, err, num_sms, st)                  \
                 : launch_tc<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st);
+  if (pair && bn == 224) {  // FFN1-shaped (8960 = 40 x 224 balances the waves)
+    if (kind == EPI_GELU && out_bf16) return launch_tc2<224, EPI_GELU, bf16>(a, b, cm, M, N, K, ep, err, num_sms, st);
+    if (kind == EPI_STORE && !out_bf16)
+      return launch_tc2<224, EPI_STORE, float>(a, b, cm, M, N, K, ep, err, num_sms, st);
+    return cudaErrorInvalidValue;
+  }
   if (out_bf16) {
     FH_TC_CASE(128, EPI_STORE, bf16)
     FH_TC_CASE(256, EPI_STORE, bf16)
