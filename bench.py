@@ -54,9 +54,9 @@ def slice_tflop() -> float:
 
 
 # launches per class inside one slice, and each launch's algorithmic flops
-CLASS_NAMES = {1: "gated-residual GEMMs: gemm_tc2_kernel<128,EPI_RESID> (CTA pair; O-proj, cross-O) and "
-                  "gemm_tc2s_kernel<256,EPI_RESID> (split-K on clusters of four; FFN2)",
-               2: "gemm_tc2_kernel<256,EPI_GELU> (CTA pair; FFN1)"}
+CLASS_NAMES = {1: "gated-residual GEMMs (O-proj, cross-O, FFN2): gemm_tc2s_kernel<256,EPI_RESID> "
+                  "(split-K on clusters of four CTAs, two cta_group::2 pairs)",
+               2: "gemm_tc2_kernel<224,EPI_GELU> (CTA pair; FFN1)"}
 
 
 def class_flops_per_launch(cls: int) -> float:
