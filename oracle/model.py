@@ -5,10 +5,10 @@ TEST INFRASTRUCTURE ONLY (see the package docstring).
 What the pages fix, and where:
   * gizai:flashhead (gizstack API reference), opening paragraph: the picture's
     reference latent is 5 frames of 16 x 16; each slice's audio becomes 5 latent
-    frames of 32 audio tokens; "a Wan-style transformer (30 blocks of 1536, 12
-    heads, its rotary over frame, row and column)" predicts the flow of the noisy
-    latent, whose first latent frames are the motion of the slice before, in 4
-    steps.
+    frames of 32 audio tokens; a Wan-style transformer of 30 blocks of width 1536
+    with 12 heads and rotary embeddings over frame, row and column predicts, in 4
+    steps, the flow of the noisy latent, whose first latent frames carry the motion
+    of the previous slice.
   * gizai:flashhead, Types > FlashHead: ``patch`` and ``head`` are Linear layers;
     ``headMods`` holds, at each step, the output norm's shift and scale [2, 1536];
     ``cos``/``sin`` are [1280, 768] with pair d of head h at column h*64 + d.
@@ -40,7 +40,10 @@ Readings where the pages are silent (the same readings bind the CUDA library):
       w_k = 10000^(-k/128); e = Linear(SiLU(Linear(sinusoid))); e0 = Linear(SiLU(e))
       gives 6 x D; block mods = table_k + e0; head mods = head table + e.
   R11 every Linear has a bias.
-  R12 sampler update is Euler x += (sigma' - sigma) v.
+  R12 sampler update is Euler x += (sigma' - sigma) v (the benchmark contract). The
+      re-noising update the audio-cpp doc names for distilled checkpoints, which it does
+      not define, is read as x0 = x - sigma v, then x = (1 - sigma') x0 + sigma' eps with
+      a fresh N(0, 1) draw eps per step (``renoise_update``, ``sample_slice_renoise``).
   R14 frames 0-1 are overwritten with the motion latent before every network call
       and once more on the output.
   R15 the initial state at sigma = 1 is the noise for frames 2-4.
@@ -434,4 +437,28 @@ def sample_slice(W: Weights, noise, ref, motion, audio, sigmas, prec):
         x = pin_motion(x, motion)
         v = predict_flow(W, x, ref, audio, sigmas[s], prec, kvs=kvs, ang=ang)
         x = (x + np.asarray(sigmas[s + 1] - sigmas[s], dtype=dt) * v).astype(dt)
+    return pin_motion(x, motion)
+
+
+def renoise_update(x, v, sigma, sigma_next, eps):
+    """One re-noising step (reading R12 of the update that SoulX-FlashHead (audio-cpp model
+    doc), Generate / Variant boundaries, names for distilled checkpoints): the flow's clean
+    estimate x0 = x - sigma v is put back on the noise path at sigma_next with fresh noise,
+    x' = (1 - sigma_next) x0 + sigma_next eps. At sigma_next = 0 it is the Euler step."""
+    dt = x.dtype
+    x0 = (x - np.asarray(sigma, dtype=dt) * v).astype(dt)
+    return (np.asarray(1.0 - sigma_next, dtype=dt) * x0 + np.asarray(sigma_next, dtype=dt) * eps).astype(dt)
+
+
+def sample_slice_renoise(W: Weights, noise, ref, motion, audio, sigmas, eps, prec):
+    """The slice sampler with the re-noising update (R12, R14, R15); eps [steps, B, C, F, H, W]
+    holds the fresh draw of each step (its frames 0..1 are overwritten by the motion pin)."""
+    dt = _dt(prec)
+    kvs = [cross_kv(W, k, audio, prec) for k in range(W.cfg.blocks)]
+    ang = rope_angles(W.cfg)
+    x = np.asarray(noise, dtype=dt)
+    for s in range(len(sigmas) - 1):
+        x = pin_motion(x, motion)
+        v = predict_flow(W, x, ref, audio, sigmas[s], prec, kvs=kvs, ang=ang)
+        x = renoise_update(x, v, sigmas[s], sigmas[s + 1], np.asarray(eps[s], dtype=dt))
     return pin_motion(x, motion)

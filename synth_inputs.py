@@ -148,6 +148,7 @@ IN_NOISE = IN_X + 3     # initial noise [B, C, F, H, W]
 IN_REF = IN_X + 4       # reference latent [B, C, F, H, W]
 IN_MOTION = IN_X + 5    # motion latent [B, C, 2, H, W]
 IN_LATENT = IN_X + 6    # noisy latent for one prediction [B, C, F, H, W]
+IN_RENOISE = IN_X + 7   # fresh noise of the re-noising sampler, one draw per step [S, B, C, F, H, W]
 
 
 def config_seed(index: int) -> int:
@@ -173,6 +174,11 @@ def latent(seed: int, tid: int, batch: int, ch: int, frames: int, h: int, w: int
 def audio_tokens(seed: int, batch: int, frames: int, tokens: int, dim: int, bf16: bool) -> np.ndarray:
     a = normal(seed, IN_AUDIO, (batch, frames, tokens, dim)).astype(np.float32)
     return to_bf16(a) if bf16 else a
+
+
+def renoise_draws(seed: int, steps: int, batch: int, ch: int, frames: int, h: int, w: int) -> np.ndarray:
+    """The fresh N(0, 1) draws of a re-noising sampler slice, [steps, B, C, F, H, W] float32."""
+    return normal(seed, IN_RENOISE, (steps, batch, ch, frames, h, w)).astype(np.float32)
 
 
 def slice_inputs(seed: int, batch: int, ch: int, frames: int, h: int, w: int,

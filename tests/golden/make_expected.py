@@ -12,6 +12,8 @@ bf16 paths):
   cfg2          one flow prediction at sigma 0.75, batch 1, 5x16x16 latent
   cfg3_s0/s19   the 4-step slice sampler, slices 0 and 19 (fresh audio per slice)
   cfg4_b0       the 4-step sampler at 5x24x24 (2880 tokens), stream 0 of the 3-stream batch
+  cfg3_renoise_s0  the 4-step slice sampler with the re-noising update (reading R12), slice 0,
+                its fresh draws from si.renoise_draws(seed of slice 0, 4, ...)
 """
 from __future__ import annotations
 
@@ -61,6 +63,13 @@ def make(case: str, W2=None):
         noise, ref, motion, audio = si.slice_inputs(seed, 1, cfg.latent_ch, cfg.frames, cfg.lat_h, cfg.lat_w,
                                                     cfg.audio_tokens, cfg.dim, True, j)
         out = om.sample_slice(W, noise, ref, motion, audio, SIGMAS, "f32")
+    elif case == "cfg3_renoise_s0":
+        cfg, seed = om.CFG3, si.config_seed(3)
+        W = W2 or om.make_weights(cfg, NET_SEED)
+        noise, ref, motion, audio = si.slice_inputs(seed, 1, cfg.latent_ch, cfg.frames, cfg.lat_h, cfg.lat_w,
+                                                    cfg.audio_tokens, cfg.dim, True, 0)
+        eps = si.renoise_draws(seed, len(SIGMAS) - 1, 1, cfg.latent_ch, cfg.frames, cfg.lat_h, cfg.lat_w)
+        out = om.sample_slice_renoise(W, noise, ref, motion, audio, SIGMAS, eps, "f32")
     elif case == "cfg4_b0":
         cfg, seed = om.CFG4, si.config_seed(4)
         base = W2 or om.make_weights(om.CFG2, NET_SEED)
@@ -75,7 +84,7 @@ def make(case: str, W2=None):
           flush=True)
 
 
-CASES = ["cfg2", "cfg3_s0", "cfg3_s19", "cfg4_b0"]
+CASES = ["cfg2", "cfg3_s0", "cfg3_s19", "cfg4_b0", "cfg3_renoise_s0"]
 
 if __name__ == "__main__":
     cases = sys.argv[1:] or CASES

@@ -328,6 +328,71 @@ def test_sampler_matches_manual_euler_steps():
     assert np.max(np.abs(out - x)) < 1e-12
 
 
+def test_renoise_with_the_current_noise_estimate_is_the_euler_step():
+    """On the linear noise path x = (1 - s) x0 + s e the velocity is v = e - x0, so the
+    noise the flow implies is e_hat = x0_hat + v. Re-noising with e_hat must land exactly
+    where the Euler step x + (s' - s) v does: a dropped term, a flipped sign or swapped
+    sigmas in the re-noising update breaks this."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((3, 7, 5))
+    v = rng.standard_normal((3, 7, 5))
+    for s, s2 in [(1.0, 0.75), (0.75, 0.5), (0.5, 0.25), (0.3, 0.0)]:
+        e_hat = (x - s * v) + v
+        got = om.renoise_update(x, v, s, s2, e_hat)
+        assert np.allclose(got, x + (s2 - s) * v, rtol=0, atol=1e-12)
+
+
+def test_renoise_with_the_exact_velocity_returns_a_fresh_point_of_the_path():
+    """For x on the path between a clean sample x0 and noise e at level s, and the exact
+    velocity e - x0, the update recovers x0 and re-noises it with the fresh draw: the
+    result is (1 - s') x0 + s' e_fresh, whatever e was."""
+    rng = np.random.default_rng(12)
+    x0, e, e_fresh = (rng.standard_normal((4, 9)) for _ in range(3))
+    for s, s2 in [(1.0, 0.75), (0.6, 0.2), (0.25, 0.0)]:
+        x = (1 - s) * x0 + s * e
+        got = om.renoise_update(x, e - x0, s, s2, e_fresh)
+        assert np.allclose(got, (1 - s2) * x0 + s2 * e_fresh, rtol=0, atol=1e-12)
+
+
+def test_renoise_sampler_single_final_step_is_euler_and_ignores_the_draw():
+    """With sigmas (s, 0) the re-noising sampler takes one step to sigma 0, which puts no
+    weight on the fresh draw: the output equals the Euler sampler's for any draw,
+    bitwise in float64, and the motion frames are the motion latent."""
+    W = om.make_weights(TINY, 31)
+    noise, ref, motion, audio = si.slice_inputs(32, 1, TINY.latent_ch, TINY.frames, TINY.lat_h, TINY.lat_w,
+                                                TINY.audio_tokens, TINY.dim, False)
+    sig = [0.6, 0.0]
+    euler = om.sample_slice(W, noise, ref, motion, audio, sig, "f64")
+    for seed in (1, 2):
+        eps = si.renoise_draws(seed, 1, 1, TINY.latent_ch, TINY.frames, TINY.lat_h, TINY.lat_w)
+        got = om.sample_slice_renoise(W, noise, ref, motion, audio, sig, eps, "f64")
+        assert np.array_equal(got, euler)
+        assert np.array_equal(got[:, :, :2], motion)
+
+
+def test_renoise_sampler_matches_manual_steps():
+    """The sampler applies the update after each network call with that step's own draw
+    (eps[s] at step s, not another step's), pinning the motion frames before each call."""
+    W = om.make_weights(TINY, 33)
+    noise, ref, motion, audio = si.slice_inputs(34, 1, TINY.latent_ch, TINY.frames, TINY.lat_h, TINY.lat_w,
+                                                TINY.audio_tokens, TINY.dim, False)
+    sig = [1.0, 0.7, 0.3, 0.0]
+    eps = si.renoise_draws(35, 3, 1, TINY.latent_ch, TINY.frames, TINY.lat_h, TINY.lat_w)
+    e64 = eps.astype(np.float64)
+    x = noise.astype(np.float64)
+    for s in range(3):
+        x = om.pin_motion(x, motion)
+        v = om.predict_flow(W, x, ref, audio, sig[s], "f64")
+        x = (1 - sig[s + 1]) * (x - sig[s] * v) + sig[s + 1] * e64[s]
+    want = om.pin_motion(x, motion)
+    got = om.sample_slice_renoise(W, noise, ref, motion, audio, sig, eps, "f64")
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+    # a different draw for the middle step changes the result
+    eps2 = eps.copy()
+    eps2[1] = -eps2[1]
+    assert not np.allclose(om.sample_slice_renoise(W, noise, ref, motion, audio, sig, eps2, "f64"), want)
+
+
 def test_predict_flow_token_order():
     """Patchify / unpatchify are inverse and use token n = f*H*W + h*W + w."""
     lat = si.normal(3, 3, (2, 4, 3, 2, 5))
