@@ -97,6 +97,7 @@ def load_library() -> ctypes.CDLL:
         "fh_dit_block_forward": (I, [P, I, P, P, P, P, I, P, P]),
         "fh_dit_predict_flow": (I, [P, P, P, P, F, P, I, P, P]),
         "fh_sample_slice": (I, [P, P, P, P, P, P, I, P, I, P, P]),
+        "fh_sample_slice_renoise": (I, [P, P, P, P, P, P, I, P, P, I, P, P]),
         "fh_sample_slice_host": (I, [P, P, P, P, P, P, I, P, I, P, P]),
         "fh_dit_get_weight": (I, [P, I, P, Z]),
         "fh_dit_sync": (I, [P, P]),
@@ -215,6 +216,16 @@ class DiT:
         _check(load_library().fh_sample_slice(self._h, _ptr(noise), _ptr(ref), _ptr(motion), _ptr(audio),
                                               _farr(sigmas), len(sigmas) - 1, _ptr(out), B, _ptr(ws),
                                               _stream(stream)))
+        return out
+
+    def sample_slice_renoise(self, noise, ref, motion, audio, sigmas, eps, ws, out=None, stream=None):
+        """The sampler with the re-noising update; eps [steps, B, C, F, H, W] float32 on the device."""
+        import torch
+        B = noise.shape[0]
+        out = torch.empty_like(noise) if out is None else out
+        _check(load_library().fh_sample_slice_renoise(self._h, _ptr(noise), _ptr(ref), _ptr(motion), _ptr(audio),
+                                                      _farr(sigmas), len(sigmas) - 1, _ptr(eps), _ptr(out), B,
+                                                      _ptr(ws), _stream(stream)))
         return out
 
     def sample_slice_host(self, noise, ref, motion, audio, sigmas, ws, out, stream=None):

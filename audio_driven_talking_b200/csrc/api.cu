@@ -174,6 +174,7 @@ struct Plan {
 
 struct GraphEntry {
   void* ws;
+  const float* eps;  // the re-noising sampler's draws (null: Euler)
   int batch, nsteps, timing;
   std::vector<float> sigmas;
   cudaGraphExec_t exec;
@@ -544,16 +545,21 @@ int run_network(fh_dit* m, Plan& P, cudaStream_t st) {
 }
 
 template <typename T>
-int run_sampler_steps(fh_dit* m, Plan& P, const float* sig, int nsteps, cudaStream_t st) {
+int run_sampler_steps(fh_dit* m, Plan& P, const float* sig, int nsteps, const float* eps, cudaStream_t st) {
   const WsLayout& w = P.lay;
   RUN(run_cross_kv(m, P, 0, m->NB, st));
+  const size_t draw = (size_t)P.batch * m->C * m->L;  // floats per step of the re-noising draws
   for (int s = 0; s < nsteps; ++s) {
     TVals tv;
     for (int b = 0; b < 8; ++b) tv.t[b] = sig[s];
     RUN(run_time_cond(m, P, tv, st));
     RUN(run_network<T>(m, P, st));
-    LAUNCH(euler_step<T>(at<float>(P.ws, w.lat), at<float>(P.ws, w.v), sig[s + 1] - sig[s], 2 * m->HW,
-                         at<T>(P.ws, w.tok), P.batch, m->C, m->L, st));
+    if (eps)
+      LAUNCH(renoise_step<T>(at<float>(P.ws, w.lat), at<float>(P.ws, w.v), eps + s * draw, sig[s], sig[s + 1],
+                             2 * m->HW, at<T>(P.ws, w.tok), P.batch, m->C, m->L, st));
+    else
+      LAUNCH(euler_step<T>(at<float>(P.ws, w.lat), at<float>(P.ws, w.v), sig[s + 1] - sig[s], 2 * m->HW,
+                           at<T>(P.ws, w.tok), P.batch, m->C, m->L, st));
   }
   return FH_OK;
 }
@@ -904,7 +910,7 @@ int fh_dit_predict_flow(fh_dit* m, const float* x_noisy, const float* ref, const
 }
 
 static int sample_impl(fh_dit* m, const float* noise, const float* ref, const float* motion, const float* sigmas,
-                       int nsteps, float* x_out, int batch, void* ws, cudaStream_t st) {
+                       int nsteps, const float* eps, float* x_out, int batch, void* ws, cudaStream_t st) {
   Plan* P;
   RUN(get_plan(m, ws, batch, &P));
   const WsLayout& w = P->lay;
@@ -919,7 +925,7 @@ static int sample_impl(fh_dit* m, const float* noise, const float* ref, const fl
   // find or record the graph of the step loop
   GraphEntry* g = nullptr;
   for (auto& e : m->graphs)
-    if (e.ws == ws && e.batch == batch && e.nsteps == nsteps && e.timing == m->timing &&
+    if (e.ws == ws && e.eps == eps && e.batch == batch && e.nsteps == nsteps && e.timing == m->timing &&
         memcmp(e.sigmas.data(), sigmas, sizeof(float) * (nsteps + 1)) == 0)
       g = &e;
   if (!g) {
@@ -932,8 +938,8 @@ static int sample_impl(fh_dit* m, const float* noise, const float* ref, const fl
     m->launches = 0;
     m->ev_used = 0;
     m->last_pairs.clear();
-    int rc = m->bf16 ? run_sampler_steps<bf16>(m, *P, sigmas, nsteps, m->cap)
-                     : run_sampler_steps<float>(m, *P, sigmas, nsteps, m->cap);
+    int rc = m->bf16 ? run_sampler_steps<bf16>(m, *P, sigmas, nsteps, eps, m->cap)
+                     : run_sampler_steps<float>(m, *P, sigmas, nsteps, eps, m->cap);
     m->capturing = false;
     cudaGraph_t graph = nullptr;
     cudaError_t ce = cudaStreamEndCapture(m->cap, &graph);
@@ -948,6 +954,7 @@ static int sample_impl(fh_dit* m, const float* noise, const float* ref, const fl
     if (ce != cudaSuccess) return fail(FH_ERR_CUDA, "graph instantiation failed: %s", cudaGetErrorString(ce));
     GraphEntry ge;
     ge.ws = ws;
+    ge.eps = eps;
     ge.batch = batch;
     ge.nsteps = nsteps;
     ge.timing = m->timing;
@@ -983,7 +990,23 @@ int fh_sample_slice(fh_dit* m, const float* noise, const float* ref, const float
   RUN(get_plan(m, ws, batch, &P));
   CK(cudaMemcpyAsync(at<void>(ws, P->lay.audio), audio, (size_t)batch * m->F * m->A * m->D * elt(m),
                      cudaMemcpyDeviceToDevice, st));
-  return sample_impl(m, noise, ref, motion, sigmas, nsteps, x_out, batch, ws, st);
+  return sample_impl(m, noise, ref, motion, sigmas, nsteps, nullptr, x_out, batch, ws, st);
+}
+
+int fh_sample_slice_renoise(fh_dit* m, const float* noise, const float* ref, const float* motion, const void* audio,
+                            const float* sigmas, int nsteps, const float* eps, float* x_out, int batch, void* ws,
+                            void* stream) {
+  RUN(common_checks(m, batch, ws));
+  RUN(check_sigmas(sigmas, nsteps));
+  if (!noise || !ref || !motion || !audio || !eps || !x_out || !aligned16(noise) || !aligned16(ref) ||
+      !aligned16(motion) || !aligned16(audio) || !aligned16(eps) || !aligned16(x_out))
+    return fail(FH_ERR_ARG, "null or unaligned pointer");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Plan* P;
+  RUN(get_plan(m, ws, batch, &P));
+  CK(cudaMemcpyAsync(at<void>(ws, P->lay.audio), audio, (size_t)batch * m->F * m->A * m->D * elt(m),
+                     cudaMemcpyDeviceToDevice, st));
+  return sample_impl(m, noise, ref, motion, sigmas, nsteps, eps, x_out, batch, ws, st);
 }
 
 int fh_sample_slice_host(fh_dit* m, const float* noise_host, const float* ref_host, const float* motion_host,
@@ -1004,7 +1027,7 @@ int fh_sample_slice_host(fh_dit* m, const float* noise_host, const float* ref_ho
                      cudaMemcpyHostToDevice, st));
   CK(cudaMemcpyAsync(at<void>(ws, w.audio), audio_host, (size_t)batch * m->F * m->A * m->D * elt(m),
                      cudaMemcpyHostToDevice, st));
-  RUN(sample_impl(m, at<float>(ws, w.in_noise), at<float>(ws, w.in_ref), at<float>(ws, w.in_motion), sigmas, nsteps,
+  RUN(sample_impl(m, at<float>(ws, w.in_noise), at<float>(ws, w.in_ref), at<float>(ws, w.in_motion), sigmas, nsteps, nullptr,
                   at<float>(ws, w.out), batch, ws, st));
   CK(cudaMemcpyAsync(x_out_host, at<void>(ws, w.out), lat, cudaMemcpyDeviceToHost, st));
   CK(cudaStreamSynchronize(st));

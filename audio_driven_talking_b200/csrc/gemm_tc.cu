@@ -5,18 +5,27 @@
 // contiguous). This is every dense contraction of the DiT: patch embed, QKV,
 // O-proj, cross-Q, cross-KV, cross-O, FFN1, FFN2 and the head.
 //
-// Design (one CTA per SM, persistent over 128 x BN output tiles):
-//   warp 0     TMA producer: one thread streams 128x64 A and BNx64 W tiles with
-//              the 128-byte swizzle into a STAGES-deep shared-memory ring
-//              (per-CTA loads; no cluster multicast).
-//   warp 1     allocates 2*BN TMEM columns and, from one thread, issues
-//              tcgen05.mma (M=128, N=BN, K=16, fp32 accumulate in TMEM); each
-//              stage is released by tcgen05.commit to its "empty" mbarrier and
-//              each finished tile by a commit to its accumulator's "full" barrier.
+// Three kernels, all warp-specialised with 192 threads:
+//   warp 0     TMA producer: one thread streams 64-deep A and W tiles with the
+//              128-byte swizzle into a STAGES-deep shared-memory ring (per-CTA
+//              loads, no cluster multicast), the first stages' W before the
+//              programmatic-launch dependency wait (W is never written).
+//   warp 1     allocates TMEM and, from one thread, issues tcgen05.mma (fp32
+//              accumulate in TMEM); each stage is released by tcgen05.commit to
+//              its "empty" mbarrier and each finished tile by a commit to its
+//              accumulator's "full" barrier.
 //   warps 2-5  epilogue: tcgen05.ld of 32 columns at a time (warp w reads TMEM
-//              lanes 32*(w%4)..+31 = its 32 output rows), the fused epilogue,
-//              direct 16-byte stores. Two accumulators alternate, so the
-//              epilogue of tile i overlaps the MMAs of tile i+1.
+//              lanes 32*(w%4)..+31 = its 32 output rows) and the fused epilogue.
+// gemm_tc_kernel    one CTA per SM, persistent over 128 x BN tiles
+//                   (cta_group::1), two accumulators so the epilogue of tile i
+//                   overlaps the MMAs of tile i+1, direct 16-byte stores.
+// gemm_tc2_kernel   a CTA pair (cluster of 2) per 256 x BN tile (cta_group::2),
+//                   persistent, two accumulators; the epilogue stages 32 x 32
+//                   boxes in shared memory and stores them by TMA (the residual
+//                   as a TMA fp32 reduce-add into x).
+// gemm_tc2s_kernel  split-K: one 256 x 256 tile per cluster of four CTAs (two
+//                   pairs, half of K each), reduce-scattered between the pairs
+//                   through shared memory, then the same staged epilogue.
 // Every wait is bounded (FH_WAIT_LIMIT_NS); on expiry the CTA latches an error
 // bit, lets the producer's in-flight copies land, frees TMEM and exits.
 #include <cstdio>

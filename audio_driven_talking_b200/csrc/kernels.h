@@ -106,6 +106,11 @@ cudaError_t prep_tokens(const float* x, const float* ref, const float* motion, i
 template <typename T>
 cudaError_t euler_step(float* lat, const float* v, float dsig, int pinned_tokens, T* tok, int batch, int C, int L,
                        cudaStream_t st);
+// the re-noising step: x0 = x - sig v, x = (1 - sig_next) x0 + sig_next eps (eps
+// channel-first [B, C, L], this step's draw), motion tokens untouched, tok refreshed.
+template <typename T>
+cudaError_t renoise_step(float* lat, const float* v, const float* eps, float sig, float sig_next, int pinned_tokens,
+                         T* tok, int batch, int C, int L, cudaStream_t st);
 cudaError_t tokens_to_latent(const float* tok, float* out, int batch, int C, int L, cudaStream_t st);
 
 // seeded weights (misc.cu): element (r, c) of tensor `tid` -> dst[r * ld + c]

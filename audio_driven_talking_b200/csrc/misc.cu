@@ -349,6 +349,32 @@ __global__ void euler_kernel(float* __restrict__ lat, const float* __restrict__ 
   }
 }
 
+// The re-noising step (reading R12 of the update the audio-cpp doc names for distilled
+// checkpoints): x0 = x - sigma v, then x = (1 - sigma') x0 + sigma' eps with this step's
+// fresh draw eps, channel-first [B, C, L]; the motion tokens (n < pinned_tokens) keep x.
+// At sigma' = 0 it computes the Euler step's fmaf(-sigma, v, x) exactly.
+template <typename T>
+__global__ void renoise_kernel(float* __restrict__ lat, const float* __restrict__ v, const float* __restrict__ eps,
+                               float sig, float sig_next, int pinned_tokens, T* __restrict__ tok, int C, int L,
+                               long total) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const float keep = 1.f - sig_next;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+    const long row = i / C;
+    const int c = (int)(i % C);
+    const int n = (int)(row % L);
+    const long b = row / L;
+    float x = lat[i];
+    if (n >= pinned_tokens) {
+      const float x0 = fmaf(-sig, v[i], x);
+      x = fmaf(sig_next, eps[(b * C + c) * L + n], keep * x0);
+      lat[i] = x;
+    }
+    tok[row * 2 * C + c] = from_f<T>(x);
+  }
+}
+
 __global__ void tokens_to_latent_kernel(const float* __restrict__ tok, float* __restrict__ out, int C, int L) {
   pdl_launch_dependents();
   pdl_wait();
@@ -617,6 +643,18 @@ cudaError_t euler_step(float* lat, const float* v, float dsig, int pinned_tokens
 }
 template cudaError_t euler_step<float>(float*, const float*, float, int, float*, int, int, int, cudaStream_t);
 template cudaError_t euler_step<bf16>(float*, const float*, float, int, bf16*, int, int, int, cudaStream_t);
+
+template <typename T>
+cudaError_t renoise_step(float* lat, const float* v, const float* eps, float sig, float sig_next, int pinned_tokens,
+                         T* tok, int batch, int C, int L, cudaStream_t st) {
+  const long n = (long)batch * L * C;
+  { cudaError_t e_ = launch_pdl(renoise_kernel<T>, dim3(grid_for(n, 256)), dim3(256), 0, st, lat, v, eps, sig, sig_next, pinned_tokens, tok, C, L, n); if (e_ != cudaSuccess) return e_; }
+  return cudaGetLastError();
+}
+template cudaError_t renoise_step<float>(float*, const float*, const float*, float, float, int, float*, int, int, int,
+                                         cudaStream_t);
+template cudaError_t renoise_step<bf16>(float*, const float*, const float*, float, float, int, bf16*, int, int, int,
+                                        cudaStream_t);
 
 cudaError_t tokens_to_latent(const float* tok, float* out, int batch, int C, int L, cudaStream_t st) {
   if (C % 32 != 0) return cudaErrorInvalidValue;

@@ -314,6 +314,26 @@ def run_gpu(args, rank, world, local_rank):
     h2d = hn.nbytes + hr.nbytes + hm.nbytes + haud[0].numel() * haud[0].element_size()
     d2h = hout.nbytes
 
+    # the re-noising sampler (reading R12 of the update for distilled checkpoints) on the
+    # same slices: one buffer of seeded draws per slice workload, refilled in place
+    eps = torch.from_numpy(si.renoise_draws(INPUT_SEED, len(SIGMAS) - 1, 1, C, F, H, W)).to(dev)
+    m.sample_slice_renoise(nd, rd, md, audios[0], SIGMAS, eps, ws, out=out)   # records its graph
+    m.sync()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(stream)
+    for j in range(K):
+        m.sample_slice_renoise(nd, rd, md, audios[j], SIGMAS, eps, ws, out=out)
+    r1.record(stream)
+    torch.cuda.synchronize()
+    m.sync()
+    tr = torch.tensor([r0.elapsed_time(r1)], device=dev)
+    if world > 1:
+        dist.all_reduce(tr, op=dist.ReduceOp.MAX)
+        dist.barrier()
+
     if rank == 0:
         frames = FRAMES_PER_SLICE * K * world
         value = frames / (ms_max / 1000.0)
@@ -334,6 +354,9 @@ def run_gpu(args, rank, world, local_rank):
                          "traffic": measured_traffic(timing_class), "launches_timed": kernel_n,
                          "mean_launch_us": kernel_us, "peak_kind": f"bf16 sustained ({src})",
                          "flops_per_launch": class_flops_per_launch(timing_class)},
+            "renoise_sampler": {"value": FRAMES_PER_SLICE * K * world / (float(tr.item()) / 1000.0), "unit": UNIT,
+                                "ms_per_step": float(tr.item()) / K,
+                                "note": "same workload, re-noising update with seeded fresh draws per step"},
             "gpu_launches": launches_per_slice * K,
             "clocks": clk.summary(),
         }

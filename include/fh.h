@@ -143,6 +143,20 @@ int fh_sample_slice(fh_dit* m, const float* noise, const float* ref, const float
                     const void* audio, const float* sigmas, int nsteps, float* x_out,
                     int batch, void* ws, void* stream);
 
+/* The slice sampler with the re-noising update that the SoulX-FlashHead audio-cpp doc
+ * (Generate / Variant boundaries) names for distilled checkpoints without defining it,
+ * read as: x0 = x - sigmas[s] v, then x = (1 - sigmas[s+1]) x0 + sigmas[s+1] eps[s].
+ * Everything else (motion pinning, inputs, outputs, graph recording) is as in
+ * fh_sample_slice; at sigmas[s+1] = 0 the step equals the Euler step exactly.
+ * eps: device float32 [nsteps, B, C, F, H, W], the fresh N(0, 1) draw of each step,
+ * caller-owned and read during the call (frames 0-1 are overwritten by the motion pin,
+ * so their values do not matter). The recorded graph is keyed on the eps pointer too:
+ * refill the same buffer between slices to replay it. Errors as fh_sample_slice;
+ * FH_ERR_ARG also for a null or unaligned eps. */
+int fh_sample_slice_renoise(fh_dit* m, const float* noise, const float* ref, const float* motion,
+                            const void* audio, const float* sigmas, int nsteps, const float* eps,
+                            float* x_out, int batch, void* ws, void* stream);
+
 /* fh_sample_slice with HOST buffers: the inputs are copied host -> device into the
  * workspace, the slice runs, and the clean latent is copied back to x_out_host;
  * returns once x_out_host is written (the stream is synchronised). Pinned host

@@ -114,6 +114,55 @@ def test_ragged_bf16_sampler_matches_oracle():
     check("ragged_432tok_b2_predict", v.cpu().numpy(), vref, TOL_BF16)
 
 
+def _renoise_case(orc, seed, batch, steps):
+    return si.renoise_draws(seed, steps, batch, orc.latent_ch, orc.frames, orc.lat_h, orc.lat_w)
+
+
+def test_ragged_bf16_renoise_sampler_matches_oracle():
+    """The re-noising sampler (reading R12) on the ragged network against the oracle's."""
+    lib, orc = _ragged()
+    m = model("ragged", lib, 77)
+    W = om.make_weights(orc, 77)
+    noise, ref, motion, audio = si.slice_inputs(78, 2, orc.latent_ch, orc.frames, orc.lat_h, orc.lat_w,
+                                                orc.audio_tokens, orc.dim, True)
+    eps = _renoise_case(orc, 79, 2, len(SIGMAS) - 1)
+    ws = m.workspace(2)
+    out = m.sample_slice_renoise(to_dev(noise), to_dev(ref), to_dev(motion), to_dev(audio, torch.bfloat16), SIGMAS,
+                                 to_dev(eps), ws)
+    m.sync()
+    got = out.cpu().numpy()
+    expect = om.sample_slice_renoise(W, noise, ref, motion, audio, SIGMAS, eps, ORACLE_PREC_BF16)
+    assert np.array_equal(got[:, :, :2], motion)
+    check("ragged_432tok_b2_renoise", got, expect, TOL_BF16)
+
+
+def test_renoise_final_step_is_the_euler_step_bitwise():
+    """A single step to sigma 0 puts no weight on the draw: the re-noising sampler's output
+    equals the Euler sampler's bit for bit, for two different draws."""
+    lib, orc = _ragged()
+    m = model("ragged", lib, 77)
+    noise, ref, motion, audio = si.slice_inputs(80, 2, orc.latent_ch, orc.frames, orc.lat_h, orc.lat_w,
+                                                orc.audio_tokens, orc.dim, True)
+    args = (to_dev(noise), to_dev(ref), to_dev(motion), to_dev(audio, torch.bfloat16))
+    sig = [0.6, 0.0]
+    ws = m.workspace(2)
+    euler = m.sample_slice(*args, sig, ws).cpu().numpy()
+    for seed in (81, 82):
+        got = m.sample_slice_renoise(*args, sig, to_dev(_renoise_case(orc, seed, 2, 1)), ws).cpu().numpy()
+        assert np.array_equal(got, euler)
+    # with more steps the draws matter
+    sig3 = [1.0, 0.5, 0.0]
+    a = m.sample_slice_renoise(*args, sig3, to_dev(_renoise_case(orc, 83, 2, 2)), ws).cpu().numpy()
+    b = m.sample_slice_renoise(*args, sig3, to_dev(_renoise_case(orc, 84, 2, 2)), ws).cpu().numpy()
+    assert not np.array_equal(a[:, :, 2:], b[:, :, 2:])
+    with pytest.raises(fh.FHError) as e:
+        lib_h = fh.load_library()
+        fh._check(lib_h.fh_sample_slice_renoise(m._h, fh._ptr(args[0]), fh._ptr(args[1]), fh._ptr(args[2]),
+                                                fh._ptr(args[3]), fh._farr(sig), 1, None, fh._ptr(args[0]), 2,
+                                                fh._ptr(ws), None))
+    assert e.value.code == fh.FH_ERR_ARG
+
+
 # ---------------------------------------------------------------------------- config 2
 def test_cfg2_predict_flow_matches_oracle():
     m = model(2)
@@ -142,6 +191,24 @@ def test_cfg3_sampler_slice_matches_oracle(slice_index):
     got = out.cpu().numpy()
     assert np.array_equal(got[:, :, :2], motion)
     check(f"cfg3_slice{slice_index}", got, expected(f"cfg3_s{slice_index}"), TOL_BF16)
+
+
+def test_cfg3_renoise_slice_matches_oracle():
+    """The re-noising sampler (reading R12) on the full-size slice, slice 0's inputs and the
+    draws si.renoise_draws(seed, 4, ...), against the stored oracle output."""
+    m = model(3)
+    ocfg = oracle_config(3)
+    seed = si.config_seed(3)
+    noise, ref, motion, audio = si.slice_inputs(seed, 1, ocfg.latent_ch, ocfg.frames, ocfg.lat_h, ocfg.lat_w,
+                                                ocfg.audio_tokens, ocfg.dim, True, 0)
+    eps = _renoise_case(ocfg, seed, 1, len(SIGMAS) - 1)
+    ws = m.workspace(1)
+    out = m.sample_slice_renoise(to_dev(noise), to_dev(ref), to_dev(motion), to_dev(audio, torch.bfloat16), SIGMAS,
+                                 to_dev(eps), ws)
+    m.sync()
+    got = out.cpu().numpy()
+    assert np.array_equal(got[:, :, :2], motion)
+    check("cfg3_renoise_slice0", got, expected("cfg3_renoise_s0"), TOL_BF16)
 
 
 def test_cfg3_host_buffer_entry_matches_device_entry():
