@@ -221,6 +221,28 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def rank_env():
+    """(world, rank, local_rank) of this process, from the variables torchrun sets (1, 0, 0 alone)."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value, world, device):
+    """The largest of every rank's `value` (a device time in ms), on every rank: the
+    job's time is its slowest replica's. Every rank must call it at the same point."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_frames_per_s(slices_per_rank, world, ms_max):
+    """Whole-job throughput: the frames every replica produced over the slowest one's time."""
+    return FRAMES_PER_SLICE * slices_per_rank * world / (ms_max / 1000.0)
+
+
 def workload_config(world, steps):
     return {"workload": "slice sampler: 4 Euler steps over 30 blocks x 1536 (12 heads x 128), latent 5x16x16 = "
                         "1280 tokens (512x512), batch 1, motion frames pinned, fresh audio per slice",
@@ -270,10 +292,7 @@ def run_gpu(args, rank, world, local_rank):
 
     with ClockSampler(local_rank) as clk:
         ms = timed(K)
-    tms = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(tms, op=dist.ReduceOp.MAX)
-    ms_max = float(tms.item())
+    ms_max = max_over_ranks(ms, world, dev)
 
     # roofline pass: the same slices again with CUDA events around every launch of one
     # kernel class (events recorded inside the graph; kept out of the headline timing)
@@ -307,9 +326,8 @@ def run_gpu(args, rank, world, local_rank):
         m.sample_slice_host(hn, hr, hm, haud[j], SIGMAS, ws, hout)
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], device=dev)
+    te_max = max_over_ranks(e0.elapsed_time(e1), world, dev)
     if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
         dist.barrier()
     h2d = hn.nbytes + hr.nbytes + hm.nbytes + haud[0].numel() * haud[0].element_size()
     d2h = hout.nbytes
@@ -329,14 +347,12 @@ def run_gpu(args, rank, world, local_rank):
     r1.record(stream)
     torch.cuda.synchronize()
     m.sync()
-    tr = torch.tensor([r0.elapsed_time(r1)], device=dev)
+    tr_max = max_over_ranks(r0.elapsed_time(r1), world, dev)
     if world > 1:
-        dist.all_reduce(tr, op=dist.ReduceOp.MAX)
         dist.barrier()
 
     if rank == 0:
-        frames = FRAMES_PER_SLICE * K * world
-        value = frames / (ms_max / 1000.0)
+        value = job_frames_per_s(K, world, ms_max)
         burst, sustained, src = peaks()
         tflops = slice_tflop() * K * world / (ms_max / 1000.0)
         achieved = class_flops_per_launch(timing_class) / (kernel_us * 1e-6) / 1e12 if kernel_n else None
@@ -346,7 +362,7 @@ def run_gpu(args, rank, world, local_rank):
             "dtype": "bf16", "data": "synthetic (seeded latents, audio tokens and weights)",
             "config": workload_config(world, K),
             "tflops": tflops, "tflops_frac_burst": tflops / burst, "peak_note": src,
-            "e2e": {"value": FRAMES_PER_SLICE * K * world / (float(te.item()) / 1000.0), "unit": UNIT,
+            "e2e": {"value": job_frames_per_s(K, world, te_max), "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
             "roofline": {"bound": "tensor", "kernel": CLASS_NAMES[timing_class], "achieved": achieved,
                          "peak": sustained, "unit": "TFLOP/s",
@@ -354,8 +370,8 @@ def run_gpu(args, rank, world, local_rank):
                          "traffic": measured_traffic(timing_class), "launches_timed": kernel_n,
                          "mean_launch_us": kernel_us, "peak_kind": f"bf16 sustained ({src})",
                          "flops_per_launch": class_flops_per_launch(timing_class)},
-            "renoise_sampler": {"value": FRAMES_PER_SLICE * K * world / (float(tr.item()) / 1000.0), "unit": UNIT,
-                                "ms_per_step": float(tr.item()) / K,
+            "renoise_sampler": {"value": job_frames_per_s(K, world, tr_max), "unit": UNIT,
+                                "ms_per_step": tr_max / K,
                                 "note": "same workload, re-noising update with seeded fresh draws per step"},
             "gpu_launches": launches_per_slice * K,
             "clocks": clk.summary(),
@@ -376,9 +392,7 @@ def main():
     ap.add_argument("--timing-class", type=int, default=1, choices=[1, 2])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local_rank = rank_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
