@@ -256,9 +256,26 @@ __global__ void gemv_kernel(const WT* __restrict__ W, const float* __restrict__ 
   float acc[8];
   for (int b = 0; b < batch; ++b) acc[b] = 0.f;
   const WT* wr = W + (long)n * K;
-  for (int k = lane; k < K; k += 32) {
-    const float wv = to_f(wr[k]);
-    for (int b = 0; b < batch; ++b) acc[b] = fmaf(wv, xs[b * K + k], acc[b]);
+  if (sizeof(WT) == 2 && K % 256 == 0) {
+    // bf16 rows: 16-byte loads, 8 weights per lane per load, two loads in flight
+#pragma unroll 2
+    for (int k0 = lane * 8; k0 < K; k0 += 256) {
+      float w8[8];
+      load8(reinterpret_cast<const bf16*>(wr) + k0, w8);
+      for (int b = 0; b < batch; ++b) {
+        const float4 x0 = *reinterpret_cast<const float4*>(xs + b * K + k0);
+        const float4 x1 = *reinterpret_cast<const float4*>(xs + b * K + k0 + 4);
+        float a = acc[b];
+        a = fmaf(w8[0], x0.x, a); a = fmaf(w8[1], x0.y, a); a = fmaf(w8[2], x0.z, a); a = fmaf(w8[3], x0.w, a);
+        a = fmaf(w8[4], x1.x, a); a = fmaf(w8[5], x1.y, a); a = fmaf(w8[6], x1.z, a); a = fmaf(w8[7], x1.w, a);
+        acc[b] = a;
+      }
+    }
+  } else {
+    for (int k = lane; k < K; k += 32) {
+      const float wv = to_f(wr[k]);
+      for (int b = 0; b < batch; ++b) acc[b] = fmaf(wv, xs[b * K + k], acc[b]);
+    }
   }
   for (int b = 0; b < batch; ++b) {
     float s = warp_sum(acc[b]);
