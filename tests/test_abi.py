@@ -69,6 +69,11 @@ def test_null_and_shape_errors_on_host(lib):
     assert lib.fh_dit_create(ctypes.byref(bad3), 0, None, ctypes.byref(out)) == fh.FH_ERR_SHAPE
     assert lib.fh_dit_sync(None, None) == fh.FH_ERR_ARG
     assert lib.fh_dit_get_weight(None, 0, None, 0) == fh.FH_ERR_ARG
+    # the samplers reject a null model before touching a device
+    sig = (ctypes.c_float * 5)(1.0, 0.75, 0.5, 0.25, 0.0)
+    assert lib.fh_sample_slice(None, None, None, None, None, sig, 4, None, 1, None, None) == fh.FH_ERR_ARG
+    assert lib.fh_sample_slice_renoise(None, None, None, None, None, sig, 4, None, None, 1, None, None) == fh.FH_ERR_ARG
+    assert b"null" in lib.fh_last_error()
 
 
 def test_no_device_is_rejected_not_substituted(lib):
