@@ -393,6 +393,25 @@ def test_renoise_sampler_matches_manual_steps():
     assert not np.allclose(om.sample_slice_renoise(W, noise, ref, motion, audio, sig, eps2, "f64"), want)
 
 
+@pytest.mark.parametrize("mistake", ["dropped_keep_factor", "swapped_sigmas", "plus_sigma_v"])
+def test_planted_renoise_mistakes_are_caught(mistake):
+    """Each plausible slip in the re-noising update, planted in a copy of it, breaks the
+    Euler identity that the pins above check."""
+    def wrong(x, v, s, s2, e):
+        if mistake == "dropped_keep_factor":
+            return (x - s * v) + s2 * e
+        if mistake == "swapped_sigmas":
+            return (1 - s) * (x - s2 * v) + s * e
+        return (1 - s2) * (x + s * v) + s2 * e
+    rng = np.random.default_rng(13)
+    x, v = rng.standard_normal((2, 6, 4))
+    s, s2 = 0.75, 0.5
+    e_hat = (x - s * v) + v
+    euler = x + (s2 - s) * v
+    assert np.allclose(om.renoise_update(x, v, s, s2, e_hat), euler, rtol=0, atol=1e-12)
+    assert not np.allclose(wrong(x, v, s, s2, e_hat), euler, rtol=0, atol=1e-6)
+
+
 def test_predict_flow_token_order():
     """Patchify / unpatchify are inverse and use token n = f*H*W + h*W + w."""
     lat = si.normal(3, 3, (2, 4, 3, 2, 5))
