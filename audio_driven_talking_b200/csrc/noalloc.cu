@@ -1,10 +1,9 @@
 // noalloc.cu - a block forward that allocates nothing, for callers that cannot allocate.
 //
 // fh_dit_block_forward needs a caller-allocated workspace. Some callers cannot call
-// cudaMalloc at the point where they run a block: code that executes while a CUDA
-// stream is being captured into a graph (an allocation there is not capturable),
-// plugins that run inside a host framework that owns all device memory, and real-time
-// threads that must not take the allocator's locks. For them this file provides
+// cudaMalloc at the point where they run a block: plugins that run inside a host
+// framework that owns all device memory, and real-time threads that must not take the
+// allocator's locks. For them this file provides
 // fh_dit_block_forward_noalloc, which runs the same kernels on a scratch buffer that
 // the library itself holds as a file-scope __device__ array (FH_STATIC_SCRATCH_BYTES;
 // every GPU that loads this library keeps it until the process exits).

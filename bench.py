@@ -150,7 +150,10 @@ class ClockSampler:
 
 class OracleSample:
     """The oracle, as it stands, on a bounded sample of the workload: whole blocks of the
-    1280-token bf16-operand network; a slice is 4 steps x 30 blocks of them."""
+    1280-token network in the oracle's plain float32 mode (the parity reference of the bf16
+    paths); a slice is 4 steps x 30 blocks of them."""
+
+    PREC = "f32"
 
     def __init__(self):
         from oracle import model as om
@@ -158,12 +161,12 @@ class OracleSample:
         cfg = om.CFG3
         self.W = om.make_weights(cfg, NET_SEED, blocks=[0, 1, 2, 3])
         self.x, self.a, t = si.block_inputs(INPUT_SEED, 1, cfg.tokens, cfg.dim, cfg.frames, cfg.audio_tokens, True)
-        _, self.e0 = om.time_conditioning(self.W, t, "bf16")
+        _, self.e0 = om.time_conditioning(self.W, t, self.PREC)
         self.ang = om.rope_angles(cfg)
         self.n = 0
 
     def block(self):
-        self.x = self.om.block_forward(self.W, self.n % 4, self.x, self.a, self.e0, "bf16", ang=self.ang)
+        self.x = self.om.block_forward(self.W, self.n % 4, self.x, self.a, self.e0, self.PREC, ang=self.ang)
         self.n += 1
 
     @staticmethod
@@ -191,13 +194,15 @@ def cpu_baseline(target_s: float = 15.0):
             break
     per_block = el / n
     return FRAMES_PER_SLICE / (per_block * 4 * NB), o.cores(), \
-        f"{n} blocks of the 1280-token network (numpy, bf16 operands), {per_block:.3f} s/block, " \
+        f"{n} blocks of the 1280-token network (numpy float32 oracle), {per_block:.3f} s/block, " \
         f"scaled x{4 * NB} blocks per slice"
 
 
 def run_reference(args, rank, world):
-    """The CPU oracle timed as the reference arm: each step is one block of the network
-    (a bounded sample of a slice), scaled to frames/s of whole slices."""
+    """The CPU oracle timed as the reference arm. Each step is ONE BLOCK of the network (a
+    bounded sample of a slice, which is 4 x 30 blocks): `steps` counts blocks and
+    `ms_per_step` is milliseconds per block; `value` is the frames/s of whole slices that
+    this block time implies, and `slice_extrapolation` states the scaling."""
     if rank != 0:
         return
     o = OracleSample()
@@ -210,12 +215,16 @@ def run_reference(args, rank, world):
     el = time.perf_counter() - t0
     per_block = el / steps
     fps = FRAMES_PER_SLICE / (per_block * 4 * NB)
-    sample = f"{steps} blocks of the 1280-token network (numpy, bf16 operands), {per_block:.3f} s/block, " \
+    sample = f"{steps} blocks of the 1280-token network (numpy float32 oracle), {per_block:.3f} s/block, " \
              f"scaled x{4 * NB} blocks per slice"
+    cfg = workload_config(1, steps)
+    cfg["step_unit"] = "one block of the network (a slice is 4 steps x 30 blocks)"
     line = {"impl": "reference", "metric": METRIC, "value": fps, "unit": UNIT, "n_gpus": args.gpus, "steps": steps,
-            "warmup": args.warmup, "ms_per_step": 1000.0 * per_block * 4 * NB, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32 (bf16-rounded operands)", "data": "synthetic",
-            "config": workload_config(1, steps),
+            "warmup": args.warmup, "ms_per_step": 1000.0 * per_block, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": cfg,
+            "slice_extrapolation": {"blocks_per_slice": 4 * NB, "ms_per_slice": 1000.0 * per_block * 4 * NB,
+                                    "frames_per_slice": FRAMES_PER_SLICE},
             "cpu_baseline": {"value": fps, "unit": UNIT, "cores": o.cores(), "kind": "oracle", "sample": sample},
             "e2e": {"value": fps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

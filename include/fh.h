@@ -188,9 +188,9 @@ int fh_dit_set_timing(fh_dit* m, int kernel_class);
 int fh_dit_get_timing(fh_dit* m, double* mean_us, int* launches);
 
 /* fh_dit_block_forward without a workspace argument, for callers that cannot allocate
- * device memory where they run a block (code running while a stream is captured into a
- * CUDA graph, plugins inside a framework that owns all device memory, real-time threads
- * that must not take allocator locks). The pages have no counterpart: this is a
+ * device memory where they run a block (plugins inside a host framework that owns all
+ * device memory, real-time threads that must not take the allocator's locks). The pages
+ * have no counterpart: this is a
  * deployment variant, not a step of the method. The scratch is a file-scope __device__
  * array of FH_STATIC_SCRATCH_BYTES (16 MiB) inside the library, held on every GPU that
  * loads the library until the process exits; calls whose fh_dit_workspace_bytes exceeds

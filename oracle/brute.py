@@ -146,3 +146,40 @@ def block_tokens(W, k, x, audio, t, tokens):
         xi = xi + g2 * _matvec(p["w2"], p["b2"], u)
         out.append(xi)
     return np.array(out)
+
+
+def predict_flow(W, x_noisy, ref, audio, sigma):
+    """Velocity [C, F, H, W] of one stream for one sigma, token by token in float64.
+
+    x_noisy, ref [C, F, H, W]; audio [F, A, D]. The steps of a flow prediction as the
+    gizai:flashhead page (opening paragraph; Types > FlashHead: ``patch``, ``head``,
+    ``headMods``) and readings R9, R10, R16 give them, written without ``oracle.model``:
+    each token's input is its noisy channels followed by its reference channels, mapped by
+    the patch Linear; the blocks are ``block_tokens`` chained over every token; the output
+    norm is an RMSNorm without gain followed by (1 + scale) and shift, where (shift, scale)
+    are the head's table rows plus the conditioning vector e of this sigma; the head Linear
+    gives the token's C velocity channels, written back to (channel, frame, row, column).
+    """
+    cfg = W.cfg
+    g = W.glob
+    C, F, H, Wd = x_noisy.shape
+    eps = cfg.eps
+    e, _ = _conditioning(W, sigma)
+    shift = np.asarray(g["head_mod"][0], dtype=np.float64) + e
+    scale = np.asarray(g["head_mod"][1], dtype=np.float64) + e
+    coords = [(f, r, c) for f in range(F) for r in range(H) for c in range(Wd)]   # token n = f*H*W + r*W + c
+    rows = []
+    for (f, r, c) in coords:
+        chans = [float(x_noisy[ch, f, r, c]) for ch in range(C)] + [float(ref[ch, f, r, c]) for ch in range(C)]
+        rows.append(_matvec(g["patch_w"], g["patch_b"], chans))
+    x = np.array(rows)
+    L = len(coords)
+    for k in range(cfg.blocks):
+        x = block_tokens(W, k, x, audio, sigma, range(L))
+    v = np.empty((C, F, H, Wd))
+    for n, (f, r, c) in enumerate(coords):
+        hn = [a * (1.0 + sc) + sh for a, sc, sh in zip(_rms(list(x[n]), eps), scale, shift)]
+        vn = _matvec(g["head_w"], g["head_b"], hn)
+        for ch in range(C):
+            v[ch, f, r, c] = vn[ch]
+    return v

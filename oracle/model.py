@@ -399,24 +399,43 @@ def unpatchify(tok, cfg: Config):
     return tok.transpose(0, 2, 1).reshape(B, C, cfg.frames, cfg.lat_h, cfg.lat_w)
 
 
+def patch_embed(W: Weights, x_noisy, ref, prec):
+    """Residual stream entering block 0: the patch Linear (gizai:flashhead, Types > FlashHead,
+    ``patch``) over each token's channels, the noisy latent's first, then the reference's (R16)."""
+    dt = _dt(prec)
+    tok = np.concatenate([patchify(x_noisy), patchify(ref)], axis=2)
+    return linear(tok.astype(dt), W.glob["patch_w"], W.glob["patch_b"], prec)
+
+
+def head_mods(W: Weights, e):
+    """Per-stream (shift, scale) of the output norm, [B, 2, D]: the head's modulation table
+    plus the conditioning vector e (reading R10; ``headMods``, gizai:flashhead, Types > FlashHead)."""
+    return W.glob["head_mod"].astype(np.float64)[None] + e[:, None, :]
+
+
+def output_head(W: Weights, x, hm, prec):
+    """Velocity tokens [B, L, C]: RMSNorm without gain, then (1 + scale) + shift (R9), then the
+    head Linear (gizai:flashhead, Types > FlashHead, ``head``)."""
+    cfg = W.cfg
+    dt = _dt(prec)
+    shift, scl = hm[:, 0, None, :], hm[:, 1, None, :]
+    hn = (rms_norm(x, cfg.eps) * (1.0 + scl) + shift).astype(dt)
+    return linear(hn, W.glob["head_w"], W.glob["head_b"], prec)
+
+
 def predict_flow(W: Weights, x_noisy, ref, audio, sigma, prec, kvs=None, ang=None):
     """v = head(RMSNorm(blocks(patch([x_noisy | ref]))) ...) for one sigma; [B, C, F, H, W]."""
     cfg = W.cfg
-    g = W.glob
     dt = _dt(prec)
     B = x_noisy.shape[0]
     if ang is None:
         ang = rope_angles(cfg)
-    tok = np.concatenate([patchify(x_noisy), patchify(ref)], axis=2)       # R16
-    x = linear(tok.astype(dt), g["patch_w"], g["patch_b"], prec)
+    x = patch_embed(W, x_noisy, ref, prec)
     e, e0 = time_conditioning(W, np.full((B,), sigma, dtype=np.float64), prec)
     for k in range(cfg.blocks):
         kv = None if kvs is None else kvs[k]
         x = block_forward(W, k, x, audio, e0, prec, ang=ang, kv=kv)
-    hm = g["head_mod"].astype(np.float64)[None] + e[:, None, :]          # [B, 2, D]
-    shift, scl = hm[:, 0, None, :], hm[:, 1, None, :]
-    hn = (rms_norm(x, cfg.eps) * (1.0 + scl) + shift).astype(dt)          # R9
-    v = linear(hn, g["head_w"], g["head_b"], prec)
+    v = output_head(W, x, head_mods(W, e), prec)
     return unpatchify(v, cfg).astype(dt)
 
 

@@ -473,3 +473,89 @@ def test_planted_cross_frame_leak_is_caught(cfg0_case, monkeypatch):
     y = _block(W, x, a, t)
     yb = brute.block_tokens(W, 0, x[0], a[0], float(t[0]), [5, 77])
     assert rel(y[0, [5, 77]], yb) > 1e-4
+
+
+# ---------------------------------------------------------------------------
+# flow prediction: patch embed, output norm with the head mods, head Linear
+# ---------------------------------------------------------------------------
+PRED = om.Config(dim=256, heads=2, ffn=512, blocks=2, latent_ch=16, frames=3, lat_h=4, lat_w=4,
+                 audio_tokens=8, bf16=False)
+PRED_SIGMA = 0.6
+
+
+@pytest.fixture(scope="module")
+def pred_case():
+    W = om.make_weights(PRED, 41)
+    noise, ref, _, audio = si.slice_inputs(42, 1, PRED.latent_ch, PRED.frames, PRED.lat_h, PRED.lat_w,
+                                           PRED.audio_tokens, PRED.dim, False)
+    vb = brute.predict_flow(W, noise[0], ref[0], audio[0], PRED_SIGMA)
+    return W, noise, ref, audio, vb
+
+
+def _pred(W, noise, ref, audio):
+    return om.predict_flow(W, noise, ref, audio, PRED_SIGMA, "f64")[0]
+
+
+def test_conditioning_matches_brute_force(pred_case):
+    W = pred_case[0]
+    e, e0 = om.time_conditioning(W, np.array([PRED_SIGMA]), "f64")
+    eb, e0b = brute._conditioning(W, PRED_SIGMA)
+    assert rel(e[0], eb) < 1e-12
+    assert rel(e0[0], e0b) < 1e-12
+
+
+def test_predict_flow_matches_float64_brute_force(pred_case):
+    """The whole prediction (patch embed over [noisy | ref], two blocks, RMSNorm with the
+    head mods = head table + e, head Linear, token order) against the per-token brute force."""
+    W, noise, ref, audio, vb = pred_case
+    assert rel(_pred(W, noise, ref, audio), vb) < 1e-10
+
+
+def _head_variant(kind):
+    """A copy of the oracle's output head with one plausible slip planted in it."""
+    def head(W, x, hm, prec):
+        dt = om._dt(prec)
+        shift, scl = hm[:, 0, None, :], hm[:, 1, None, :]
+        if kind == "layer_norm":
+            hn = om.layer_norm(x, W.cfg.eps) * (1.0 + scl) + shift
+        elif kind == "dropped_one":
+            hn = om.rms_norm(x, W.cfg.eps) * scl + shift
+        elif kind == "swapped_shift_scale":
+            hn = om.rms_norm(x, W.cfg.eps) * (1.0 + shift) + scl
+        elif kind == "shift_before_norm":
+            hn = om.rms_norm(x + shift, W.cfg.eps) * (1.0 + scl)
+        else:
+            raise ValueError(kind)
+        return om.linear(hn.astype(dt), W.glob["head_w"], W.glob["head_b"], prec)
+    return head
+
+
+@pytest.mark.parametrize("kind", ["layer_norm", "dropped_one", "swapped_shift_scale", "shift_before_norm"])
+def test_planted_output_head_mistakes_are_caught(pred_case, monkeypatch, kind):
+    W, noise, ref, audio, vb = pred_case
+    monkeypatch.setattr(om, "output_head", _head_variant(kind))
+    assert rel(_pred(W, noise, ref, audio), vb) > 1e-4
+
+
+def test_planted_reversed_concat_is_caught(pred_case, monkeypatch):
+    W, noise, ref, audio, vb = pred_case
+
+    def ref_first(W_, x_noisy, ref_, prec):
+        tok = np.concatenate([om.patchify(ref_), om.patchify(x_noisy)], axis=2)
+        return om.linear(tok.astype(om._dt(prec)), W_.glob["patch_w"], W_.glob["patch_b"], prec)
+
+    monkeypatch.setattr(om, "patch_embed", ref_first)
+    assert rel(_pred(W, noise, ref, audio), vb) > 1e-4
+
+
+def test_planted_e0_for_e_in_head_mods_is_caught(pred_case, monkeypatch):
+    """The head mods taking the block conditioning e0 (its first row) instead of e."""
+    W, noise, ref, audio, vb = pred_case
+    orig = om.time_conditioning
+
+    def e0_as_e(W_, t, prec):
+        e, e0 = orig(W_, t, prec)
+        return e0[:, 0, :].copy(), e0
+
+    monkeypatch.setattr(om, "time_conditioning", e0_as_e)
+    assert rel(_pred(W, noise, ref, audio), vb) > 1e-4

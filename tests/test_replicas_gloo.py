@@ -83,6 +83,12 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_zero():
     line = lines[0]
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+    # a step is one block: the timed work is steps x ms_per_step, and the slice figure is
+    # stated apart as the extrapolation it is
+    ex = line["slice_extrapolation"]
+    assert line["steps"] == 1 and ex["blocks_per_slice"] == 120
+    assert abs(ex["ms_per_slice"] - 120 * line["ms_per_step"]) < 1e-6 * ex["ms_per_slice"]
+    assert abs(line["value"] - 24 / (ex["ms_per_slice"] / 1000.0)) < 1e-9 * line["value"]
 
 
 def _replica_that_dies(index, world, port, out_dir):

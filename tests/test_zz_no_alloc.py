@@ -2,15 +2,15 @@
 workspace entry point it mirrors.
 
 This entry point is for callers that cannot allocate device memory where they run a
-block (stream capture into a CUDA graph, plugins inside a framework that owns all
-device memory, real-time threads). It runs on a static scratch array inside the
-library; these tests check, through the C ABI, that two calls in a row give what
-fh_dit_block_forward gives with a caller-allocated workspace, and that a model too
-large for the static scratch is refused with a clear error. The file sorts last so
-a run that stops at the first failure has run every other test first; it also
-passes alone in a fresh process.
+block (plugins inside a host framework that owns all device memory, real-time threads
+that must not take the allocator's locks). It runs the same kernels on a static
+scratch array inside the library; these tests check, through the C ABI, that two
+calls in a row give bitwise what fh_dit_block_forward gives with a caller-allocated
+workspace (the kernels are deterministic, so any difference is stale or overlapping
+scratch), and that a model too large for the static scratch is refused with a clear
+error. The file sorts last so a run that stops at the first failure has run every
+other test first; it also passes alone in a fresh process.
 """
-import numpy as np
 import pytest
 
 import synth_inputs as si
@@ -21,22 +21,14 @@ pytestmark = [pytest.mark.gpu,
 
 import audio_driven_talking_b200 as fh  # noqa: E402
 
-TOL_F32, TOL_BF16 = 1e-4, 2e-2
-
-
-def _rel(a, b):
-    a = a.double().cpu().numpy()
-    b = b.double().cpu().numpy()
-    return float(np.max(np.abs(a - b)) / np.sqrt(np.mean(b * b)))
-
 
 @pytest.mark.parametrize("which", ["fp32_block", "bf16_small"])
 def test_noalloc_block_matches_workspace_entry_twice(which):
     if which == "fp32_block":
-        cfg, tol, adt = fh.FP32_BLOCK, TOL_F32, torch.float32
+        cfg, adt = fh.FP32_BLOCK, torch.float32
     else:
         cfg = fh.ModelConfig(dim=384, heads=3, ffn=1024, blocks=2, frames=3, lat_h=12, lat_w=12)
-        tol, adt = TOL_BF16, torch.bfloat16
+        adt = torch.bfloat16
     m = fh.DiT(cfg, seed=21)
     assert 0 < m.workspace_bytes(1) <= 16 << 20
     x, a, t = si.block_inputs(22, 1, cfg.tokens, cfg.dim, cfg.frames, cfg.audio_tokens, cfg.dtype == fh.FH_BF16)
@@ -45,10 +37,11 @@ def test_noalloc_block_matches_workspace_entry_twice(which):
     k = cfg.blocks - 1
     ref = m.block_forward(k, xd, ad, list(t), ws)
     m.sync()
+    assert torch.isfinite(ref).all() and not torch.equal(ref, xd)
     for _ in range(2):
         got = m.block_forward_noalloc(k, xd, ad, list(t))
         m.sync()
-        assert _rel(got, ref) < tol
+        assert torch.equal(got, ref)
     m.close()
 
 
