@@ -183,3 +183,37 @@ def predict_flow(W, x_noisy, ref, audio, sigma):
         for ch in range(C):
             v[ch, f, r, c] = vn[ch]
     return v
+
+
+def audio_tokens(AW, states, cfg, a):
+    """Audio tokens [F, tokens, D] of one stream, in float64, frame by frame.
+
+    states [S, layers, channels]. Written without ``oracle.model``: for latent frame j the
+    video frames it covers are listed (frame 0 alone; frames 8j - 7 .. 8j after it), each
+    video frame t contributes the states within two of its position S - nv + t, the union
+    of those positions is taken in increasing order and each is clamped into [0, S - 1];
+    the selected states, flattened state by state, go through proj1 (frame 0) or proj1vf,
+    a ReLU, proj2, a ReLU and proj3, and each of the 32 tokens through a LayerNorm with
+    projNorm's weight and bias.
+    """
+    S = states.shape[0]
+    F = cfg.frames
+    nv = 1 + a.stride * (F - 1)
+    half = a.window // 2
+    out = np.empty((F, a.tokens, cfg.dim))
+    for j in range(F):
+        frames = [0] if j == 0 else list(range(a.stride * j - a.stride + 1, a.stride * j + 1))
+        pos = sorted({S - nv + t + d for t in frames for d in range(-half, half + 1)})
+        vec = []
+        for p in pos:
+            p = min(max(p, 0), S - 1)
+            vec.extend(float(v) for v in np.asarray(states[p], dtype=np.float64).reshape(-1))
+        w, b = (AW["proj1_w"], AW["proj1_b"]) if j == 0 else (AW["proj1vf_w"], AW["proj1vf_b"])
+        h = [max(0.0, v) for v in _matvec(w, b, vec)]
+        h = [max(0.0, v) for v in _matvec(AW["proj2_w"], AW["proj2_b"], h)]
+        t = _matvec(AW["proj3_w"], AW["proj3_b"], h)
+        for n in range(a.tokens):
+            tok = list(t[n * cfg.dim:(n + 1) * cfg.dim])
+            ln = _layer_norm(tok, cfg.eps)
+            out[j, n] = [v * g + c for v, g, c in zip(ln, AW["projnorm_w"], AW["projnorm_b"])]
+    return out

@@ -48,6 +48,9 @@ Readings where the pages are silent (the same readings bind the CUDA library):
       and once more on the output.
   R15 the initial state at sigma = 1 is the noise for frames 2-4.
   R16 patch input channels: the noisy latent's 128 first, then the reference's 128.
+  R19-R21 the audio projection (``audio_projection``): which encoder states each latent
+      frame reads, and proj1 / proj1vf / proj2 / proj3 / projNorm as a ReLU MLP and a
+      LayerNorm; stated where the functions are defined.
 
 Precision modes (``prec``):
   'f64'  everything in float64 (used by the pins against the brute force);
@@ -481,3 +484,99 @@ def sample_slice_renoise(W: Weights, noise, ref, motion, audio, sigmas, eps, pre
         v = predict_flow(W, x, ref, audio, sigmas[s], prec, kvs=kvs, ang=ang)
         x = renoise_update(x, v, sigmas[s], sigmas[s + 1], np.asarray(eps[s], dtype=dt))
     return pin_motion(x, motion)
+
+
+# ---------------------------------------------------------------------------
+# audio projection: speech-encoder states -> the latent frames' audio tokens
+# ---------------------------------------------------------------------------
+# gizai:flashhead, opening paragraph: for each slice the last 8 s of speech go through
+# wav2vec 2.0 base, its 12 layers' states taken at 200 frames, and 5 states around each of
+# the slice's 33 frames make 5 latent frames of 32 audio tokens; Types > FlashHead lists the
+# projection as proj1, proj1vf, proj2, proj3 (Linear layers) and projNorm (tensors).
+# Readings (the pages give no widths or formulas):
+#   R19 the slice's video frames are the last of the 200 states: video frame t (of 33)
+#       sits at state 200 - 33 + t; its 5 states are that one and two either side,
+#       indices clamped to [0, 199].
+#   R20 33 = 1 + 4 x 8 (the video VAE's temporal stride 8): latent frame 0 is video frame 0
+#       alone; latent frame j >= 1 is video frames 8j - 7 .. 8j, whose 5-state windows
+#       together span 12 consecutive states.
+#   R21 latent frame 0: a = relu(proj1(its 5 states x 12 layers x 768, state-major));
+#       later frames: a = relu(proj1vf(their 12 states x 12 x 768)); then
+#       b = relu(proj2(a)), 32 tokens of width D from proj3(b), and projNorm a LayerNorm
+#       with learned affine (weight, bias) over each token, eps as R2. Hidden width 512.
+@dataclass(frozen=True)
+class AudioConfig:
+    states: int = 200       # encoder frames in the 8 s window
+    layers: int = 12
+    channels: int = 768
+    window: int = 5         # states around each video frame
+    stride: int = 8         # video frames per latent frame after the first
+    hidden: int = 512
+    tokens: int = 32
+
+    def video_frames(self, latent_frames: int) -> int:
+        return 1 + self.stride * (latent_frames - 1)
+
+    def group_states(self) -> int:
+        return self.stride + self.window - 1
+
+
+AUDIO = AudioConfig()
+
+AUDIO_SLOTS = [
+    (0, "proj1_w", lambda c, a: (a.hidden, a.window * a.layers * a.channels), "lin",
+     lambda c, a: a.window * a.layers * a.channels),
+    (1, "proj1_b", lambda c, a: (a.hidden,), "lin", lambda c, a: a.window * a.layers * a.channels),
+    (2, "proj1vf_w", lambda c, a: (a.hidden, a.group_states() * a.layers * a.channels), "lin",
+     lambda c, a: a.group_states() * a.layers * a.channels),
+    (3, "proj1vf_b", lambda c, a: (a.hidden,), "lin", lambda c, a: a.group_states() * a.layers * a.channels),
+    (4, "proj2_w", lambda c, a: (a.hidden, a.hidden), "lin", lambda c, a: a.hidden),
+    (5, "proj2_b", lambda c, a: (a.hidden,), "lin", lambda c, a: a.hidden),
+    (6, "proj3_w", lambda c, a: (a.tokens * c.dim, a.hidden), "lin", lambda c, a: a.hidden),
+    (7, "proj3_b", lambda c, a: (a.tokens * c.dim,), "lin", lambda c, a: a.hidden),
+    (8, "projnorm_w", lambda c, a: (c.dim,), "gain", lambda c, a: c.dim),
+    (9, "projnorm_b", lambda c, a: (c.dim,), "lnb", lambda c, a: c.dim),
+]
+AUDIO_BASE = 32   # audio projection tensors: tid = GLOBAL_BASE + AUDIO_BASE + slot
+
+
+def make_audio_weights(cfg: Config, seed: int, a: AudioConfig = AUDIO) -> dict:
+    """The audio projection's synthetic weights (bf16-rounded matrices for bf16 configs)."""
+    return {name: si.weight_value(seed, global_tid(AUDIO_BASE + slot), shp(cfg, a), kind, fan(cfg, a), cfg.dim,
+                                  cfg.bf16)
+            for slot, name, shp, kind, fan in AUDIO_SLOTS}
+
+
+def audio_windows(states, latent_frames: int, a: AudioConfig = AUDIO):
+    """(first [B, window, layers, channels], later [B, F-1, group_states, layers, channels]):
+    the states each latent frame's projection reads (R19, R20)."""
+    nv = a.video_frames(latent_frames)
+    s0 = a.states - nv                       # state of video frame 0
+    half = a.window // 2
+    idx0 = np.clip(np.arange(s0 - half, s0 + half + 1), 0, a.states - 1)
+    first = states[:, idx0]
+    later = []
+    for j in range(1, latent_frames):
+        lo = s0 + a.stride * j - (a.stride - 1) - half
+        idx = np.clip(np.arange(lo, lo + a.group_states()), 0, a.states - 1)
+        later.append(states[:, idx])
+    return first, np.stack(later, axis=1)
+
+
+def audio_projection(AW: dict, states, cfg: Config, prec, a: AudioConfig = AUDIO):
+    """Audio tokens [B, F, tokens, D] from the speech-encoder states [B, states, layers,
+    channels] (R19-R21). The projection's activations stay float32 in the bf16 mode too (its
+    weights are bf16 values); the tokens it returns are what the blocks' cross-attention reads."""
+    prec = "f32" if prec == "bf16" else prec
+    dt = _dt(prec)
+    B = states.shape[0]
+    F = cfg.frames
+    first, later = audio_windows(np.asarray(states, dtype=dt), F, a)
+    h0 = linear(first.reshape(B, -1), AW["proj1_w"], AW["proj1_b"], prec)              # [B, hidden]
+    hv = linear(later.reshape(B * (F - 1), -1), AW["proj1vf_w"], AW["proj1vf_b"], prec)
+    h = np.concatenate([h0[:, None], hv.reshape(B, F - 1, -1)], axis=1)                # [B, F, hidden]
+    h = np.maximum(h, 0).astype(dt)
+    h = np.maximum(linear(h.reshape(B * F, -1), AW["proj2_w"], AW["proj2_b"], prec), 0).astype(dt)
+    t = linear(h, AW["proj3_w"], AW["proj3_b"], prec).reshape(B, F, a.tokens, cfg.dim)
+    y = layer_norm(t, cfg.eps) * AW["projnorm_w"].astype(np.float64) + AW["projnorm_b"].astype(np.float64)
+    return y.astype(dt)

@@ -149,6 +149,7 @@ IN_REF = IN_X + 4       # reference latent [B, C, F, H, W]
 IN_MOTION = IN_X + 5    # motion latent [B, C, 2, H, W]
 IN_LATENT = IN_X + 6    # noisy latent for one prediction [B, C, F, H, W]
 IN_RENOISE = IN_X + 7   # fresh noise of the re-noising sampler, one draw per step [S, B, C, F, H, W]
+IN_STATES = IN_X + 8    # speech-encoder states of the audio window [B, frames, layers, channels]
 
 
 def config_seed(index: int) -> int:
@@ -189,3 +190,10 @@ def slice_inputs(seed: int, batch: int, ch: int, frames: int, h: int, w: int,
     motion = latent(seed, IN_MOTION, batch, ch, 2, h, w)
     audio = audio_tokens(seed + slice_index, batch, frames, audio_tokens_per_frame, dim, bf16)
     return noise, ref, motion, audio
+
+
+def speech_states(seed: int, batch: int, frames: int = 200, layers: int = 12, channels: int = 768) -> np.ndarray:
+    """Synthetic stand-in for the speech encoder's hidden states over one audio window,
+    [B, frames, layers, channels] float32 N(0, 1) (8 s at 25 states/s of a 12-layer,
+    768-wide encoder in the pages' pipeline)."""
+    return normal(seed, IN_STATES, (batch, frames, layers, channels)).astype(np.float32)

@@ -559,3 +559,103 @@ def test_planted_e0_for_e_in_head_mods_is_caught(pred_case, monkeypatch):
 
     monkeypatch.setattr(om, "time_conditioning", e0_as_e)
     assert rel(_pred(W, noise, ref, audio), vb) > 1e-4
+
+
+# ---------------------------------------------------------------------------
+# audio projection (readings R19-R21)
+# ---------------------------------------------------------------------------
+ACFG = om.Config(dim=256, heads=2, ffn=512, blocks=1, frames=5, lat_h=2, lat_w=2, bf16=False)
+AUD = om.AudioConfig(states=60, layers=3, channels=16, hidden=24, tokens=4)
+
+
+@pytest.fixture(scope="module")
+def audio_case():
+    AW = om.make_audio_weights(ACFG, 51, AUD)
+    st = si.speech_states(52, 2, AUD.states, AUD.layers, AUD.channels)
+    yb = brute.audio_tokens(AW, st[1], ACFG, AUD)
+    return AW, st, yb
+
+
+def test_audio_page_facts():
+    """33 video frames per slice make 5 latent frames (1 + 4 x 8); the last video frame is the
+    last of the 200 encoder states, 8 s at 25 per second; 5 states per video frame."""
+    facts = json.load(open(GOLDEN))
+    a = om.AUDIO
+    assert a.video_frames(om.CFG3.frames) == facts["decoded_frames_per_slice"]["value"]
+    assert a.states == facts["speech_encoder_states"]["value"]
+    assert a.states == facts["audio_window_s"]["value"] * facts["fps"]["value"]
+    assert a.layers == facts["speech_encoder_layers"]["value"]
+    assert a.window == facts["states_per_video_frame"]["value"]
+    assert a.tokens == om.CFG3.audio_tokens
+    first, later = om.audio_windows(np.arange(a.states, dtype=np.float64).reshape(1, a.states, 1, 1), 5)
+    assert list(first.reshape(-1)) == [165, 166, 167, 168, 169]
+    assert later.shape[1:3] == (4, 12)
+    assert list(later[0, 3].reshape(-1)) == [190, 191, 192, 193, 194, 195, 196, 197, 198, 199, 199, 199]
+
+
+def test_audio_projection_matches_float64_brute_force(audio_case):
+    AW, st, yb = audio_case
+    y = om.audio_projection(AW, st, ACFG, "f64", AUD)
+    assert y.shape == (2, ACFG.frames, AUD.tokens, ACFG.dim)
+    assert rel(y[1], yb) < 1e-10
+
+
+def test_audio_projection_zero_proj3_gives_the_norm_bias(audio_case):
+    """A token of zeros normalises to zero, so the output is projNorm's bias."""
+    AW, st, _ = audio_case
+    AW2 = dict(AW, proj3_w=np.zeros_like(AW["proj3_w"]), proj3_b=np.zeros_like(AW["proj3_b"]))
+    y = om.audio_projection(AW2, st, ACFG, "f64", AUD)
+    assert np.max(np.abs(y - AW["projnorm_b"].astype(np.float64))) < 1e-12
+
+
+def test_audio_projection_reads_only_its_window(audio_case):
+    """States before every window change nothing; a state near the end changes only the latent
+    frames whose windows hold it (frames 3 and 4 of 5 for the state two before the last)."""
+    AW, st, _ = audio_case
+    y = om.audio_projection(AW, st, ACFG, "f64", AUD)
+    nv = AUD.video_frames(ACFG.frames)
+    st2 = st.copy()
+    st2[:, :AUD.states - nv - 2] += 3.0
+    assert np.array_equal(om.audio_projection(AW, st2, ACFG, "f64", AUD), y)
+    st3 = st.copy()
+    st3[:, AUD.states - 3] += 1.0
+    y3 = om.audio_projection(AW, st3, ACFG, "f64", AUD)
+    assert np.array_equal(y3[:, :3], y[:, :3])
+    assert np.max(np.abs(y3[:, 3:] - y[:, 3:])) > 1e-6
+
+
+def _audio_variant(kind):
+    """A copy of the oracle's projection with one plausible slip planted in it."""
+    def windows(states, F, a=om.AUDIO):
+        nv = a.video_frames(F)
+        s0 = a.states - nv + (1 if kind == "window_off_by_one" else 0)
+        half = a.window // 2
+        first = states[:, np.clip(np.arange(s0 - half, s0 + half + 1), 0, a.states - 1)]
+        later = []
+        for j in range(1, F):
+            lo = s0 + a.stride * j - (0 if kind == "group_shift" else a.stride - 1) - half
+            later.append(states[:, np.clip(np.arange(lo, lo + a.group_states()), 0, a.states - 1)])
+        return first, np.stack(later, axis=1)
+
+    def proj(AW, states, cfg, prec, a=om.AUDIO):
+        B, F = states.shape[0], cfg.frames
+        first, later = windows(np.asarray(states, dtype=np.float64), F, a)
+        h0 = om.linear(first.reshape(B, -1), AW["proj1_w"], AW["proj1_b"], "f64")
+        hv = om.linear(later.reshape(B * (F - 1), -1), AW["proj1vf_w"], AW["proj1vf_b"], "f64")
+        h = np.concatenate([h0[:, None], hv.reshape(B, F - 1, -1)], axis=1)
+        act = (lambda v: v) if kind == "no_relu" else (lambda v: np.maximum(v, 0))
+        h = act(h)
+        h = act(om.linear(h.reshape(B * F, -1), AW["proj2_w"], AW["proj2_b"], "f64"))
+        t = om.linear(h, AW["proj3_w"], AW["proj3_b"], "f64").reshape(B, F, a.tokens, cfg.dim)
+        y = om.layer_norm(t, cfg.eps)
+        if kind != "norm_without_affine":
+            y = y * AW["projnorm_w"] + AW["projnorm_b"]
+        return y
+    return proj
+
+
+@pytest.mark.parametrize("kind", ["window_off_by_one", "group_shift", "no_relu", "norm_without_affine"])
+def test_planted_audio_projection_mistakes_are_caught(audio_case, kind):
+    AW, st, yb = audio_case
+    y = _audio_variant(kind)(AW, st, ACFG, "f64", AUD)
+    assert rel(y[1], yb) > 1e-4
