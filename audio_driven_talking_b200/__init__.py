@@ -100,6 +100,7 @@ def load_library() -> ctypes.CDLL:
         "fh_sample_slice_renoise": (I, [P, P, P, P, P, P, I, P, P, I, P, P]),
         "fh_sample_slice_host": (I, [P, P, P, P, P, P, I, P, I, P, P]),
         "fh_dit_get_weight": (I, [P, I, P, Z]),
+        "fh_audio_project": (I, [P, P, P, I, P, P]),
         "fh_dit_sync": (I, [P, P]),
         "fh_dit_last_launch_count": (I, [P]),
         "fh_dit_set_timing": (I, [P, I]),
@@ -109,6 +110,10 @@ def load_library() -> ctypes.CDLL:
         "fh_dit_block_forward_noalloc": (I, [P, I, P, P, P, P, I, P]),
         "fh_dit_probe_wait_timeout": (I, [P, P]),
         "fh_op_attention": (I, [P, P, P, P, P, I, I, I, F, I, P]),
+        "fh_op_cross_attention": (I, [P, P, P, P, P, I, I, I, I, I, F, I, P]),
+        "fh_op_row_norm": (I, [P, P, I, I, I, P, P, ctypes.c_long, I, F, I, P]),
+        "fh_op_linear_streamk_bytes": (Z, [I, I, I]),
+        "fh_op_linear_streamk": (I, [P, P, P, P, I, I, I, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -236,6 +241,17 @@ class DiT:
                                                    out.data_ptr(), B, _ptr(ws), _stream(stream)))
         return out
 
+    def audio_project(self, states, ws, out=None, stream=None):
+        """Audio tokens [B, frames, 32, dim] (model dtype) from speech-encoder states
+        [B, 200, 12, 768] float32 on the device (see include/fh.h, fh_audio_project)."""
+        import torch
+        B = states.shape[0]
+        c = self.cfg
+        if out is None:
+            out = torch.empty((B, c.frames, c.audio_tokens, c.dim), dtype=self.model_dtype, device=states.device)
+        _check(load_library().fh_audio_project(self._h, _ptr(states), _ptr(out), B, _ptr(ws), _stream(stream)))
+        return out
+
     def sync(self, stream=None):
         _check(load_library().fh_dit_sync(self._h, _stream(stream)))
 
@@ -274,6 +290,46 @@ def linear(A, W, bias, stream=None):
     return out
 
 
+def linear_streamk(A, W, bias, stream=None):
+    """linear() for bf16 CTA-pair shapes with the stream-K split of the model's block GEMMs."""
+    import torch
+    M, K = A.shape
+    N = W.shape[0]
+    lib = load_library()
+    n = int(lib.fh_op_linear_streamk_bytes(M, N, K))
+    if n == 0:
+        raise FHError(FH_ERR_SHAPE, f"bad GEMM shape {M} x {N} x {K}")
+    ws = torch.empty(n, dtype=torch.uint8, device=A.device)
+    out = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    _check(lib.fh_op_linear_streamk(_ptr(A), _ptr(W), _ptr(bias), _ptr(out), M, N, K, _ptr(ws), n, _stream(stream)))
+    return out
+
+
+def cross_attention(q, ssq_q, kv, ssq_k, frames, eps=1e-6, stream=None):
+    """Per-frame audio cross-attention (see include/fh_ops.h): q [B, frames*hw, heads*128],
+    kv [B, frames, 32, 2*heads*128] (keys then values), ssq_q/ssq_k float32 per-head sums."""
+    import torch
+    B, L, D = q.shape
+    A = kv.shape[2]
+    dt = FH_BF16 if q.dtype == torch.bfloat16 else FH_F32
+    out = torch.empty_like(q)
+    _check(load_library().fh_op_cross_attention(_ptr(q), _ptr(ssq_q), _ptr(kv), _ptr(ssq_k), _ptr(out), B, D // 128,
+                                                frames, L // frames, A, ctypes.c_float(eps), dt, _stream(stream)))
+    return out
+
+
+def row_norm(x, mode, a, c, bstride=0, rows_per_batch=None, out_dtype=None, eps=1e-6, out=None, stream=None):
+    """Row norm and modulation (see include/fh_ops.h, fh_op_row_norm): x float32 [M, D]."""
+    import torch
+    M, D = x.shape
+    out_dtype = out_dtype or torch.bfloat16
+    dt = FH_BF16 if out_dtype == torch.bfloat16 else FH_F32
+    out = torch.empty((M, D), dtype=out_dtype, device=x.device) if out is None else out
+    _check(load_library().fh_op_row_norm(_ptr(x), _ptr(out), M, D, mode, _ptr(a), _ptr(c), int(bstride),
+                                         rows_per_batch or M, ctypes.c_float(eps), dt, _stream(stream)))
+    return out
+
+
 def attention(q, k, v, ssq, eps=1e-6, stream=None):
     """Self-attention with full-width RMS factors from ssq (see include/fh_ops.h)."""
     import torch
@@ -286,4 +342,4 @@ def attention(q, k, v, ssq, eps=1e-6, stream=None):
 
 
 __all__ = ["DiT", "ModelConfig", "LITE", "FP32_BLOCK", "ONE_BLOCK", "LITE_768_X3", "FHError", "load_library",
-           "linear", "attention", "FH_F32", "FH_BF16"]
+           "linear", "linear_streamk", "attention", "cross_attention", "row_norm", "FH_F32", "FH_BF16"]

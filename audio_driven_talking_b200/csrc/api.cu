@@ -8,9 +8,11 @@
 // headMods, the [1280, 768] rotary tables and the `work: Scratch` arena, which here
 // is the caller-owned workspace; Methods > talk runs slice by slice. The launch
 // sequence of one block is the Wan-style adaLN block of readings R1-R11.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -121,28 +123,41 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Tile shape per GEMM, from the weight's N and K. Deep projections (K >= 1024, N >= 1536:
 // QKV, O-proj, cross-Q/O, FFN1, FFN2) run as 256-row tiles on CTA pairs (cta_group::2),
-// each CTA streaming half of the W tile; the rest (patch embed K=256, head N=128, the
-// per-slice cross-KV with 160 rows) on single CTAs. Tile width 224 for FFN1, 256 for the
-// cross-KV and the width-1536 projections (split-K on clusters of four at 1280 tokens), 128
-// for QKV (measured on B200 at 1280 tokens).
+// each CTA streaming half of the W tile, 256 columns wide where N allows (the widest tile
+// a pair accumulates, the least operand traffic per MMA), with a stream-K split of the
+// k-blocks over all CTA pairs so that no round of tiles runs part-empty; the rest (patch
+// embed K = 256, head N = 128, the per-slice cross-KV with 160 rows) on single CTAs.
 struct TileCfg {
   int bn;
   bool pair;
-  int wbox;  // rows of the W tile each CTA loads
+  bool streamk;  // split the k-blocks over every CTA pair (else whole tiles per pair)
+  int wbox;      // rows of the W tile each CTA loads
 };
 TileCfg tile_cfg(int N, int K, bool pair_ok = true) {
   TileCfg t;
   t.pair = pair_ok && K >= 1024 && N >= 1536 && N <= 16384;
-  // 256 wide for FFN1 and the cross-KV, and for the pair GEMMs of width up to 4096 (O-proj,
-  // cross-Q/O, FFN2), which then run split-K on clusters of four when their 256 x 256 tiles
-  // are few (kernels.h); 128 for QKV
+  // 256 wide for the cross-KV (single CTAs) and for the pair GEMMs of width up to 4096
+  // (O-proj, cross-Q/O, FFN2), which then run split-K on clusters of four when their 256 x 256
+  // tiles are few; 128 for QKV
   t.bn = (N % 256 == 0 && (N >= 8192 || (t.pair && N <= 4096))) ? 256 : 128;
   // FFN1 (N = 8960 = 40 x 224): at 1280 tokens 200 pair tiles of width 224 fill three rounds
   // of 74 CTA pairs better than 175 tiles of width 256
   if (t.pair && N >= 8192 && N % 224 == 0) t.bn = 224;
+  t.streamk = false;
   t.wbox = t.pair ? t.bn / 2 : t.bn;
   return t;
 }
+
+// The audio projection's fixed sizes: the speech encoder's window (8 s at 25 states/s, 12
+// layers of 768, wav2vec 2.0 base), 5 states per video frame, 8 video frames per latent
+// frame after the first, hidden width 512 (readings of gizai:flashhead's opening paragraph).
+constexpr int AU_STATES = 200, AU_LAYERS = 12, AU_CH = 768, AU_WIN = 5, AU_STRIDE = 8, AU_HID = 512;
+constexpr int AU_PER_STATE = AU_LAYERS * AU_CH;
+constexpr int AU_GROUP = AU_STRIDE + AU_WIN - 1;
+constexpr int AU_K0 = AU_WIN * AU_PER_STATE, AU_KV = AU_GROUP * AU_PER_STATE;
+
+constexpr bool kFuseNorms = false;  // norm of the finished rows inside the gated-residual GEMM
+constexpr int LN_COUNTERS = 8192;  // fused-norm launches per call (a 64-step slice of 30 blocks needs 5760)
 
 struct TensorRec {
   int tid;
@@ -161,7 +176,8 @@ struct BlockW {
 
 struct WsLayout {
   size_t x, h, qkv, ssq_qk, attn, cq, ssq_cq, ckv, ssq_ckv, u, tok, lat, v, mods, hmods, tsin, thid, te, te0, audio,
-      in_noise, in_ref, in_motion, out, total;
+      in_noise, in_ref, in_motion, out, sk_part, sk_flags, sk_flags_bytes, ln_ctr, au_win0, au_winv, au_part, au_h1, au_h2,
+      au_tok, total;
 };
 
 struct Plan {
@@ -170,6 +186,7 @@ struct Plan {
   WsLayout lay{};
   CUtensorMap m_h, m_attn, m_u, m_tok, m_audio, m_q, m_k, m_v;
   CUtensorMap m_xq, m_xkv, m_xo;  // cross-attention: queries and output per frame, keys/values
+  CUtensorMap m_skp;              // stream-K partial-sum slots of the CTA-pair GEMMs
 };
 
 struct GraphEntry {
@@ -199,6 +216,9 @@ struct fh_dit {
   float *patch_b = nullptr, *head_b = nullptr, *head_mod = nullptr, *t_b1 = nullptr, *t_b2 = nullptr,
         *t_bp = nullptr;
   float2* rope = nullptr;
+  // audio projection: proj1 [HID, K0], proj1vf [HID, KV], proj2 [HID, HID], proj3 [32 D, HID]
+  void *a_w1 = nullptr, *a_w1v = nullptr, *a_w2 = nullptr, *a_w3 = nullptr;
+  float *a_b1 = nullptr, *a_b1v = nullptr, *a_b2 = nullptr, *a_b3 = nullptr, *a_nw = nullptr, *a_nb = nullptr;
   CUtensorMap m_ckv_all, m_patch, m_head;
   std::vector<TensorRec> recs;
   unsigned* err_host = nullptr;
@@ -207,6 +227,7 @@ struct fh_dit {
   std::vector<GraphEntry> graphs;
   cudaStream_t cap = nullptr;
   int launches = 0, last_launches = 0;
+  int ln_seq = 0;  // fused-norm counters used so far in this call
   // timing of one kernel class inside the sampler graph
   int timing = 0;
   std::vector<cudaEvent_t> events;
@@ -218,6 +239,13 @@ struct fh_dit {
 namespace {
 
 size_t elt(const fh_dit* m) { return m->bf16 ? 2 : 4; }
+
+// whether any of the block's GEMMs runs on CTA pairs (and so needs the stream-K buffers)
+bool uses_pair_gemms(const fh_dit* m) {
+  if (!m->bf16) return false;
+  const int D = m->D, FF = m->FF;
+  return tile_cfg(3 * D, D).pair || tile_cfg(D, D).pair || tile_cfg(FF, D).pair || tile_cfg(D, FF).pair;
+}
 
 WsLayout layout(const fh_dit* m, int B) {
   WsLayout w{};
@@ -252,8 +280,41 @@ WsLayout layout(const fh_dit* m, int B) {
   w.in_ref = take((size_t)B * m->C * m->L * 4);
   w.in_motion = take((size_t)B * m->C * 2 * m->HW * 4);
   w.out = take((size_t)B * m->C * m->L * 4);
+  // audio projection: the gathered states, split-K partial sums, hidden rows, fp32 tokens
+  {
+    const size_t R = (size_t)B * m->F, HID = AU_HID, TN = (size_t)m->A * m->D;
+    w.au_win0 = take((size_t)B * AU_K0 * 4);
+    w.au_winv = take((size_t)B * (m->F - 1) * AU_KV * 4);
+    size_t part = (size_t)audio_gemv_chunks(AU_K0) * B * HID;
+    part = std::max(part, (size_t)audio_gemv_chunks(AU_KV) * B * (m->F - 1) * HID);
+    part = std::max(part, R * std::max(HID, TN));
+    w.au_part = take(part * 4);
+    w.au_h1 = take(R * HID * 4);
+    w.au_h2 = take(R * HID * 4);
+    w.au_tok = take(R * TN * 4);
+  }
+  // stream-K partial sums of the CTA-pair GEMMs: one slot of 2 x 128 rows x 256 fp32 per
+  // cluster (one per CTA pair of the GPU), and per-(tile, CTA, 32-row quarter) counters
+  // and one counter per launch of the gated-residual GEMM that normalises the rows it finished
+  // (LN_COUNTERS per call); counters and flags sit together and start every call at zero
+  w.sk_part = w.sk_flags = w.sk_flags_bytes = w.ln_ctr = 0;
+  if (uses_pair_gemms(m)) {
+    const size_t tiles = ((M + 255) / 256) * (size_t)((std::max(3 * m->D, m->FF) + 127) / 128);
+    w.sk_part = take((size_t)(m->num_sms / 2) * 2 * 128 * 256 * 4);
+    const size_t flags = al256(tiles * 2 * 4 * 4);
+    w.sk_flags = take(flags + LN_COUNTERS * 4);
+    w.ln_ctr = w.sk_flags + flags;
+    w.sk_flags_bytes = flags + LN_COUNTERS * 4;
+  }
   w.total = o;
   return w;
+}
+
+// the stream-K flags and the norm counters start every call at zero (stream-K owners also
+// clear their flags as they go)
+cudaError_t clear_sk_flags(const WsLayout& w, void* ws, cudaStream_t st) {
+  if (!w.sk_flags_bytes) return cudaSuccess;
+  return cudaMemsetAsync(reinterpret_cast<uint8_t*>(ws) + w.sk_flags, 0, w.sk_flags_bytes, st);
 }
 
 template <typename P>
@@ -287,6 +348,10 @@ int get_plan(fh_dit* m, void* ws, int B, Plan** out) {
     ok = ok && make_map_3d(&p.m_xq, at<void>(ws, w.cq), m->D, HW, frames, 64, 128) &&
          make_map_3d(&p.m_xo, at<void>(ws, w.attn), m->D, HW, frames, 64, 32) &&
          make_map(&p.m_xkv, at<void>(ws, w.ckv), frames * m->A, (uint64_t)m->NB * 2 * m->D, 32);
+    if (ok && w.sk_flags_bytes) {
+      const uint64_t rows = (uint64_t)(m->num_sms / 2) * 256;
+      ok = make_out_map(&p.m_skp, at<void>(ws, w.sk_part), rows, 256, 256, true);
+    }
     if (!ok) {
       p.ws = nullptr;
       return fail(FH_ERR_CUDA, "tensor map encoding failed for the workspace");
@@ -311,9 +376,19 @@ void timed_end(fh_dit* m, int i, cudaStream_t st) {
   m->last_pairs.push_back(i);
 }
 
+// The norm a gated-residual GEMM may apply to the rows it finished (rownorm.cuh): mode, the
+// scale / weight vector a, the shift / bias vector c, and a's and c's stride per stream.
+struct NormSpec {
+  int mode;
+  const float* a;
+  const float* c;
+  long bstride;
+};
+
 int run_gemm(fh_dit* m, const CUtensorMap* amap, const void* A, long lda, const CUtensorMap* bmap, const void* W,
              long ldw, int M, int N, int K, int kind, bool out_bf16, const EpiParams& ep, cudaStream_t st,
-             int tclass) {
+             int tclass, const NormSpec* norm = nullptr, void* norm_out = nullptr, bool* normed = nullptr) {
+  if (normed) *normed = false;
   const int ti = timed_begin(m, tclass, st);
   cudaError_t e;
   if (m->bf16) {
@@ -323,8 +398,28 @@ int run_gemm(fh_dit* m, const CUtensorMap* amap, const void* A, long lda, const 
       timed_end(m, ti, st);
       return fail(FH_ERR_CUDA, "tensor map encoding failed for a GEMM output");
     }
-    e = gemm_tc(*amap, *bmap, tc.pair ? &cmap : nullptr, M, N, K, tc.bn, kind, out_bf16, ep, m->err_dev,
-                m->num_sms, st, tc.pair);
+    EpiParams epk = ep;
+    const WsLayout& w = m->plan.lay;
+    const bool sk = tc.pair && tc.streamk && w.sk_flags_bytes;
+    if (sk) {  // stream-K over every CTA pair
+      epk.sk_part = at<float>(m->plan.ws, w.sk_part);
+      epk.sk_flags = at<int>(m->plan.ws, w.sk_flags);
+    }
+    if (tc.pair && w.sk_flags_bytes) {
+      // the next norm of the updated rows, in the same launch (width 1536, a counter left)
+      if (kFuseNorms && norm && kind == EPI_RESID && N == 12 * 128 && m->ln_seq < LN_COUNTERS) {
+        epk.ln_out = norm_out;
+        epk.ln_mode = norm->mode;
+        epk.ln_a = norm->a;
+        epk.ln_c = norm->c;
+        epk.ln_bstride = norm->bstride;
+        epk.ln_eps = m->cfg.eps;
+        epk.ln_ctr = at<int>(m->plan.ws, w.ln_ctr) + m->ln_seq++;
+        if (normed) *normed = true;
+      }
+    }
+    e = gemm_tc(*amap, *bmap, tc.pair ? &cmap : nullptr, sk ? &m->plan.m_skp : nullptr, M, N, K, tc.bn, kind,
+                out_bf16, epk, m->err_dev, m->num_sms, st, tc.pair);
   }
   else
     e = gemm_simt(reinterpret_cast<const float*>(A), lda, reinterpret_cast<const float*>(W), ldw, M, N, K, kind,
@@ -404,8 +499,13 @@ int run_cross_kv(fh_dit* m, Plan& P, int k0, int nb, cudaStream_t st) {
                   m->bf16, ep, st, 0);
 }
 
+// One block on the residual x. h_ready: the block's first norm (LN1 and its modulation) is
+// already in h (the previous block's FFN2 wrote it). after: the norm that follows the block
+// (the next block's LN1, or the output norm), which the block's last GEMM applies to the rows
+// it finishes when it can; *after_done says whether it did.
 template <typename T>
-int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
+int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec* after, bool* after_done,
+              cudaStream_t st) {
   const WsLayout& w = P.lay;
   void* ws = P.ws;
   const int B = P.batch, L = m->L, D = m->D, NH = m->NH;
@@ -418,9 +518,10 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
   T* qkv = at<T>(ws, w.qkv);
   float* ssq_qk = at<float>(ws, w.ssq_qk);
   const float eps = m->cfg.eps;
+  if (after_done) *after_done = false;
 
   // self-attention branch
-  {
+  if (!h_ready) {
     const int ti = timed_begin(m, 6, st);
     cudaError_t e = norm_rows<T>(x, h, M, D, L, 0, mods + 0 * D, mods + 1 * D, mbs, nullptr, nullptr, eps, st);
     timed_end(m, ti, st);
@@ -436,6 +537,15 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
     ep.norm_period = 3 * D;
     ep.norm_count = 2 * D;
     ep.rope = m->rope;
+    {
+      const int pf = m->cfg.rope_split[0] / 2, ph = m->cfg.rope_split[1] / 2;
+      ep.rope_H = m->cfg.lat_h;
+      ep.rope_W = m->cfg.lat_w;
+      ep.rope_pf = pf;
+      ep.rope_ph = ph;
+      ep.rope_off_h = m->F * pf;
+      ep.rope_off_w = m->F * pf + m->cfg.lat_h * ph;
+    }
     ep.dim = D;
     ep.sec_stride = (long)M * D;
     RUN(run_gemm(m, &P.m_h, h, D, &bw.m_qkv, bw.wqkv, D, M, 3 * D, D, EPI_QKV, m->bf16, ep, st, 3));
@@ -451,17 +561,21 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
     timed_end(m, ti, st);
     LAUNCH(e);
   }
+  bool normed = false;
   {
+    // O-proj + gated residual, then the learned-affine LayerNorm before the cross-attention (R7)
     EpiParams ep = epi0(L);
     ep.bias = bw.bo;
     ep.resid = x;
     ep.ldr = D;
     ep.gate = mods + 2 * D;
     ep.gate_bstride = mbs;
-    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_o, bw.wo, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1));
+    const NormSpec ln3{1, bw.ln3w, bw.ln3b, 0};
+    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_o, bw.wo, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1, &ln3, h,
+                 &normed));
   }
   // audio cross-attention branch
-  LAUNCH(norm_rows<T>(x, h, M, D, L, 1, nullptr, nullptr, 0, bw.ln3w, bw.ln3b, eps, st));
+  if (!normed) LAUNCH(norm_rows<T>(x, h, M, D, L, 1, nullptr, nullptr, 0, bw.ln3w, bw.ln3b, eps, st));
   {
     EpiParams ep = epi0(L);
     ep.bias = bw.bcq;
@@ -487,14 +601,17 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
     LAUNCH(e);
   }
   {
+    // cross-O + residual, then the FFN's LayerNorm and modulation
     EpiParams ep = epi0(L);
     ep.bias = bw.bco;
     ep.resid = x;
     ep.ldr = D;
-    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_co, bw.wco, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1));
+    const NormSpec ln2{0, mods + 4 * D, mods + 3 * D, mbs};
+    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_co, bw.wco, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1, &ln2, h,
+                 &normed));
   }
   // FFN branch
-  LAUNCH(norm_rows<T>(x, h, M, D, L, 0, mods + 3 * D, mods + 4 * D, mbs, nullptr, nullptr, eps, st));
+  if (!normed) LAUNCH(norm_rows<T>(x, h, M, D, L, 0, mods + 3 * D, mods + 4 * D, mbs, nullptr, nullptr, eps, st));
   {
     EpiParams ep = epi0(L);
     ep.bias = bw.b1;
@@ -510,7 +627,7 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
     ep.gate = mods + 5 * D;
     ep.gate_bstride = mbs;
     RUN(run_gemm(m, &P.m_u, at<T>(ws, w.u), m->FF, &bw.m_2, bw.w2, m->FF, M, D, m->FF, EPI_RESID, m->bf16, ep, st,
-                 1));
+                 1, after, h, after_done));
   }
   return FH_OK;
 }
@@ -531,9 +648,17 @@ int run_network(fh_dit* m, Plan& P, cudaStream_t st) {
     RUN(run_gemm(m, &P.m_tok, at<T>(ws, w.tok), 2 * C, &m->m_patch, m->patch_w, 2 * C, M, D, 2 * C, EPI_STORE,
                  false, ep, st, 0));
   }
-  for (int k = 0; k < m->NB; ++k) RUN(run_block<T>(m, P, k, x, st));
   float* hm = at<float>(ws, w.hmods);
-  LAUNCH(norm_rows<T>(x, at<T>(ws, w.h), M, D, L, 2, hm, hm + D, 2L * D, nullptr, nullptr, m->cfg.eps, st));
+  const long mbs = (long)m->NB * 6 * D;
+  bool h_ready = false;
+  for (int k = 0; k < m->NB; ++k) {
+    // after block k: the next block's LN1 with its modulation, or the output RMSNorm (R9)
+    const float* nm = at<float>(ws, w.mods) + (long)(k + 1) * 6 * D;
+    const NormSpec next = k + 1 < m->NB ? NormSpec{0, nm + D, nm, mbs} : NormSpec{2, hm + D, hm, 2L * D};
+    RUN(run_block<T>(m, P, k, x, h_ready, &next, &h_ready, st));
+  }
+  if (!h_ready)
+    LAUNCH(norm_rows<T>(x, at<T>(ws, w.h), M, D, L, 2, hm, hm + D, 2L * D, nullptr, nullptr, m->cfg.eps, st));
   {
     EpiParams ep = epi0(L);
     ep.bias = m->head_b;
@@ -583,16 +708,20 @@ int common_checks(fh_dit* m, int batch, void* ws) {
 }
 
 // kernels with more than 48 KB of dynamic shared memory need an attribute set per device,
-// outside any stream capture
+// outside any stream capture; done once per device (ordinals below 64), under a lock so that
+// first calls from several threads do not race on it
+std::mutex g_prepare_mu;
+bool g_prepared[64] = {};
 int prepare_device(int dev) {
-  static unsigned done = 0;
-  if (dev < 32 && (done & (1u << dev))) return FH_OK;
+  if (dev < 0 || dev >= 64) return fail(FH_ERR_UNSUPPORTED, "device ordinal %d outside [0, 64)", dev);
+  std::lock_guard<std::mutex> lock(g_prepare_mu);
+  if (g_prepared[dev]) return FH_OK;
   cudaError_t e = gemm_tc_prepare();
   if (e == cudaSuccess) e = attn_tc_prepare();
   if (e == cudaSuccess) e = cross_attn_prepare();
   if (e == cudaSuccess) e = xattn_tc_prepare();
   if (e != cudaSuccess) return fail(FH_ERR_CUDA, "kernel attribute setup: %s", cudaGetErrorString(e));
-  if (dev < 32) done |= 1u << dev;
+  g_prepared[dev] = true;
   return FH_OK;
 }
 
@@ -679,7 +808,12 @@ int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** ou
                o_mod = take(NB * 6 * D * 4), o_pw = take(D * 2 * C * e), o_pb = take(D * 4), o_hw = take(C * D * e),
                o_hb = take(C * 4), o_hm = take(2 * D * 4), o_tw1 = take(D * 256 * e), o_tb1 = take(D * 4),
                o_tw2 = take(D * D * e), o_tb2 = take(D * 4), o_twp = take(6 * D * D * e), o_tbp = take(6 * D * 4),
-               o_rope = take((size_t)L * 64 * 8);
+               o_rope = take((size_t)(c.frames + c.lat_h + c.lat_w) * 64 * 8);
+  const size_t o_aw1 = take((size_t)AU_HID * AU_K0 * e), o_ab1 = take(AU_HID * 4),
+               o_aw1v = take((size_t)AU_HID * AU_KV * e), o_ab1v = take(AU_HID * 4),
+               o_aw2 = take((size_t)AU_HID * AU_HID * e), o_ab2 = take(AU_HID * 4),
+               o_aw3 = take((size_t)32 * D * AU_HID * e), o_ab3 = take((size_t)32 * D * 4), o_anw = take(D * 4),
+               o_anb = take(D * 4);
   m->arena_bytes = off;
   if (cudaMalloc(&m->arena, off) != cudaSuccess) {
     cudaGetLastError();
@@ -723,6 +857,16 @@ int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** ou
   m->t_wp = a + o_twp;
   m->t_bp = (float*)(a + o_tbp);
   m->rope = (float2*)(a + o_rope);
+  m->a_w1 = a + o_aw1;
+  m->a_b1 = (float*)(a + o_ab1);
+  m->a_w1v = a + o_aw1v;
+  m->a_b1v = (float*)(a + o_ab1v);
+  m->a_w2 = a + o_aw2;
+  m->a_b2 = (float*)(a + o_ab2);
+  m->a_w3 = a + o_aw3;
+  m->a_b3 = (float*)(a + o_ab3);
+  m->a_nw = (float*)(a + o_anw);
+  m->a_nb = (float*)(a + o_anb);
 
   // ---- tensor records: id -> storage (the id scheme of fh.h)
   auto rec = [&](int tid, void* p, long rows, long cols, long ld, bool mat, int kind, int fan) {
@@ -773,6 +917,16 @@ int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** ou
   rec(FH_GLOBAL_TENSOR(8), m->t_b2, 1, D, D, false, LIN, (int)D);
   rec(FH_GLOBAL_TENSOR(9), m->t_wp, 6 * D, D, D, true, LIN, (int)D);
   rec(FH_GLOBAL_TENSOR(10), m->t_bp, 1, 6 * D, 6 * D, false, LIN, (int)D);
+  rec(FH_AUDIO_TENSOR(0), m->a_w1, AU_HID, AU_K0, AU_K0, true, LIN, AU_K0);
+  rec(FH_AUDIO_TENSOR(1), m->a_b1, 1, AU_HID, AU_HID, false, LIN, AU_K0);
+  rec(FH_AUDIO_TENSOR(2), m->a_w1v, AU_HID, AU_KV, AU_KV, true, LIN, AU_KV);
+  rec(FH_AUDIO_TENSOR(3), m->a_b1v, 1, AU_HID, AU_HID, false, LIN, AU_KV);
+  rec(FH_AUDIO_TENSOR(4), m->a_w2, AU_HID, AU_HID, AU_HID, true, LIN, AU_HID);
+  rec(FH_AUDIO_TENSOR(5), m->a_b2, 1, AU_HID, AU_HID, false, LIN, AU_HID);
+  rec(FH_AUDIO_TENSOR(6), m->a_w3, 32 * D, AU_HID, AU_HID, true, LIN, AU_HID);
+  rec(FH_AUDIO_TENSOR(7), m->a_b3, 1, 32 * D, 32 * D, false, LIN, AU_HID);
+  rec(FH_AUDIO_TENSOR(8), m->a_nw, 1, D, D, false, GAIN, 1);
+  rec(FH_AUDIO_TENSOR(9), m->a_nb, 1, D, D, false, LNB, 1);
 
   // ---- generate
   int rc = FH_OK;
@@ -863,7 +1017,9 @@ int fh_dit_block_forward(fh_dit* m, int block, const float* x_in, float* x_out, 
   Plan* P;
   RUN(get_plan(m, ws, batch, &P));
   m->launches = 0;
+  m->ln_seq = 0;
   const size_t M = (size_t)batch * m->L;
+  CK(clear_sk_flags(P->lay, ws, st));
   CK(cudaMemcpyAsync(at<void>(ws, P->lay.audio), audio, (size_t)batch * m->F * m->A * m->D * elt(m),
                      cudaMemcpyDeviceToDevice, st));
   if (x_out != x_in) CK(cudaMemcpyAsync(x_out, x_in, M * m->D * 4, cudaMemcpyDeviceToDevice, st));
@@ -872,9 +1028,9 @@ int fh_dit_block_forward(fh_dit* m, int block, const float* x_in, float* x_out, 
   RUN(run_cross_kv(m, *P, block, 1, st));
   RUN(run_time_cond(m, *P, tv, st));
   if (m->bf16)
-    RUN(run_block<bf16>(m, *P, block, x_out, st));
+    RUN(run_block<bf16>(m, *P, block, x_out, false, nullptr, nullptr, st));
   else
-    RUN(run_block<float>(m, *P, block, x_out, st));
+    RUN(run_block<float>(m, *P, block, x_out, false, nullptr, nullptr, st));
   m->last_launches = m->launches;
   return FH_OK;
 }
@@ -889,7 +1045,9 @@ int fh_dit_predict_flow(fh_dit* m, const float* x_noisy, const float* ref, const
   Plan* P;
   RUN(get_plan(m, ws, batch, &P));
   m->launches = 0;
+  m->ln_seq = 0;
   const WsLayout& w = P->lay;
+  CK(clear_sk_flags(w, ws, st));
   CK(cudaMemcpyAsync(at<void>(ws, w.audio), audio, (size_t)batch * m->F * m->A * m->D * elt(m),
                      cudaMemcpyDeviceToDevice, st));
   TVals tv;
@@ -936,6 +1094,7 @@ static int sample_impl(fh_dit* m, const float* noise, const float* ref, const fl
     CK(cudaStreamBeginCapture(m->cap, cudaStreamCaptureModeRelaxed));
     m->capturing = true;
     m->launches = 0;
+    m->ln_seq = 0;
     m->ev_used = 0;
     m->last_pairs.clear();
     int rc = m->bf16 ? run_sampler_steps<bf16>(m, *P, sigmas, nsteps, eps, m->cap)
@@ -965,6 +1124,7 @@ static int sample_impl(fh_dit* m, const float* noise, const float* ref, const fl
     m->graphs.push_back(ge);
     g = &m->graphs.back();
   }
+  CK(clear_sk_flags(w, ws, st));
   CK(cudaGraphLaunch(g->exec, st));
   m->last_pairs = g->ev_pairs;
   m->launches = outside + g->launches;
@@ -1032,6 +1192,53 @@ int fh_sample_slice_host(fh_dit* m, const float* noise_host, const float* ref_ho
   CK(cudaMemcpyAsync(x_out_host, at<void>(ws, w.out), lat, cudaMemcpyDeviceToHost, st));
   CK(cudaStreamSynchronize(st));
   return check_err_word(m);
+}
+
+int fh_audio_project(fh_dit* m, const float* states, void* tokens, int batch, void* ws, void* stream) {
+  RUN(common_checks(m, batch, ws));
+  if (!states || !tokens || !aligned16(states) || !aligned16(tokens)) return fail(FH_ERR_ARG, "null or unaligned pointer");
+  const int nv = 1 + AU_STRIDE * (m->F - 1);
+  if (nv > AU_STATES || m->A != 32) return fail(FH_ERR_SHAPE, "%d latent frames need %d video frames of states", m->F, nv);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Plan* P;
+  RUN(get_plan(m, ws, batch, &P));
+  const WsLayout& w = P->lay;
+  m->launches = 0;
+  const int B = batch, F = m->F, R = B * F, D = m->D;
+  float *win0 = at<float>(ws, w.au_win0), *winv = at<float>(ws, w.au_winv), *part = at<float>(ws, w.au_part),
+        *h1 = at<float>(ws, w.au_h1), *h2 = at<float>(ws, w.au_h2), *tk = at<float>(ws, w.au_tok);
+  LAUNCH(audio_windows(states, win0, winv, B, AU_STATES, AU_PER_STATE, F, AU_STATES - nv, AU_WIN, AU_STRIDE, AU_GROUP,
+                       st));
+  cudaError_t e;
+  if (m->bf16) {
+    e = audio_linear<bf16>((const bf16*)m->a_w1, win0, m->a_b1, part, h1, AU_HID, AU_K0, B, 1, 1, F, 0, st);
+    if (e == cudaSuccess)
+      e = audio_linear<bf16>((const bf16*)m->a_w1v, winv, m->a_b1v, part, h1, AU_HID, AU_KV, B * (F - 1), 1, F - 1, F,
+                             1, st);
+    if (e == cudaSuccess)
+      e = audio_linear<bf16>((const bf16*)m->a_w2, h1, m->a_b2, part, h2, AU_HID, AU_HID, R, 1, R, 0, 0, st);
+    if (e == cudaSuccess)
+      e = audio_linear<bf16>((const bf16*)m->a_w3, h2, m->a_b3, part, tk, 32 * D, AU_HID, R, 0, R, 0, 0, st);
+    if (e == cudaSuccess)
+      e = norm_rows<bf16>(tk, (bf16*)tokens, R * 32, D, R * 32, 1, nullptr, nullptr, 0, m->a_nw, m->a_nb, m->cfg.eps,
+                          st);
+  } else {
+    e = audio_linear<float>((const float*)m->a_w1, win0, m->a_b1, part, h1, AU_HID, AU_K0, B, 1, 1, F, 0, st);
+    if (e == cudaSuccess)
+      e = audio_linear<float>((const float*)m->a_w1v, winv, m->a_b1v, part, h1, AU_HID, AU_KV, B * (F - 1), 1, F - 1,
+                              F, 1, st);
+    if (e == cudaSuccess)
+      e = audio_linear<float>((const float*)m->a_w2, h1, m->a_b2, part, h2, AU_HID, AU_HID, R, 1, R, 0, 0, st);
+    if (e == cudaSuccess)
+      e = audio_linear<float>((const float*)m->a_w3, h2, m->a_b3, part, tk, 32 * D, AU_HID, R, 0, R, 0, 0, st);
+    if (e == cudaSuccess)
+      e = norm_rows<float>(tk, (float*)tokens, R * 32, D, R * 32, 1, nullptr, nullptr, 0, m->a_nw, m->a_nb, m->cfg.eps,
+                           st);
+  }
+  if (e != cudaSuccess) return fail(FH_ERR_CUDA, "audio projection launch: %s", cudaGetErrorString(e));
+  m->launches += 9;  // four split-K products with their reductions, and the norm
+  m->last_launches = m->launches;
+  return FH_OK;
 }
 
 int fh_dit_get_weight(const fh_dit* m, int tensor_id, void* host_dst, size_t bytes) {
@@ -1125,7 +1332,7 @@ int fh_op_linear(const void* A, const void* W, const float* bias, float* out, in
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     RUN(prepare_device(dev));
-    e = gemm_tc(ma, mb, &mc, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, tc.pair);
+    e = gemm_tc(ma, mb, &mc, nullptr, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, tc.pair);
   } else if (dtype == FH_F32) {
     if (K % 32) return fail(FH_ERR_SHAPE, "K %% 32 != 0");
     e = gemm_simt((const float*)A, K, (const float*)W, K, M, N, K, EPI_STORE, ep, st);
@@ -1133,6 +1340,106 @@ int fh_op_linear(const void* A, const void* W, const float* bias, float* out, in
     return fail(FH_ERR_ARG, "bad dtype");
   }
   if (e != cudaSuccess) return fail(FH_ERR_CUDA, "linear launch: %s", cudaGetErrorString(e));
+  return FH_OK;
+}
+
+size_t fh_op_linear_streamk_bytes(int M, int N, int K) {
+  if (M < 1 || N < 128 || N % 128 || K < 64 || K % 64) return 0;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const size_t tiles = ((size_t)(M + 255) / 256) * (size_t)(N / 128);
+  return al256((size_t)(sms / 2) * 256 * 256 * 4) + al256(tiles * 8 * 4);
+}
+
+int fh_op_linear_streamk(const void* A, const void* W, const float* bias, float* out, int M, int N, int K, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (!A || !W || !bias || !out || !ws || !aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255))
+    return fail(FH_ERR_ARG, "null or unaligned pointer");
+  if (M < 1 || N % 128 || K % 64) return fail(FH_ERR_SHAPE, "bad GEMM shape %d x %d x %d", M, N, K);
+  const TileCfg tc = tile_cfg(N, K);
+  if (!tc.pair) return fail(FH_ERR_SHAPE, "shape %d x %d x %d does not run on CTA pairs", M, N, K);
+  const size_t need = fh_op_linear_streamk_bytes(M, N, K);
+  if (ws_bytes < need) return fail(FH_ERR_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+  if (!load_encode()) return fail(FH_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled unavailable");
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  RUN(prepare_device(dev));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t part_bytes = al256((size_t)(sms / 2) * 256 * 256 * 4);
+  EpiParams ep = epi0(1 << 30);
+  ep.bias = bias;
+  ep.out = out;
+  ep.ldo = N;
+  ep.sk_part = reinterpret_cast<float*>(ws);
+  ep.sk_flags = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ws) + part_bytes);
+  CUtensorMap ma, mb, mc, mp;
+  if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, W, N, K, tc.wbox) || !make_out_map(&mc, out, M, N, N, true) ||
+      !make_out_map(&mp, ws, (uint64_t)(sms / 2) * 256, 256, 256, true))
+    return fail(FH_ERR_CUDA, "tensor map encoding");
+  CK(cudaMemsetAsync(ep.sk_flags, 0, need - part_bytes, st));
+  const cudaError_t e = gemm_tc(ma, mb, &mc, &mp, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, true);
+  if (e != cudaSuccess) return fail(FH_ERR_CUDA, "linear launch: %s", cudaGetErrorString(e));
+  return FH_OK;
+}
+
+int fh_op_cross_attention(const void* q, const float* ssq_q, const void* kv, const float* ssq_k, void* out, int batch,
+                          int heads, int frames, int hw, int audio_tokens, float eps, int dtype, void* stream) {
+  if (!q || !ssq_q || !kv || !ssq_k || !out || !aligned16(q) || !aligned16(kv) || !aligned16(out))
+    return fail(FH_ERR_ARG, "null or unaligned pointer");
+  if (batch < 1 || heads < 1 || heads > 64 || frames < 1 || hw < 1 || audio_tokens != 32)
+    return fail(FH_ERR_SHAPE, "bad cross-attention shape (audio_tokens must be 32)");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int D = heads * 128, L = frames * hw;
+  cudaError_t e;
+  if (dtype == FH_BF16) {
+    if (!load_encode()) return fail(FH_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled unavailable");
+    const uint64_t nf = (uint64_t)batch * frames;
+    CUtensorMap mq, mkv, mo;
+    if (!make_map_3d(&mq, q, D, hw, nf, 64, 128) || !make_map_3d(&mo, out, D, hw, nf, 64, 32) ||
+        !make_map(&mkv, kv, nf * audio_tokens, 2 * (uint64_t)D, 32))
+      return fail(FH_ERR_CUDA, "tensor map encoding");
+    int dev = 0;
+    cudaGetDevice(&dev);
+    RUN(prepare_device(dev));
+    e = xattn_tc(mq, mkv, mo, ssq_q, ssq_k, heads, 0, 0, D, batch, heads, L, frames, audio_tokens, eps, nullptr, st);
+  } else if (dtype == FH_F32) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    RUN(prepare_device(dev));
+    e = cross_attn<float>((const float*)q, ssq_q, (const float*)kv, 2L * D, 0, D, ssq_k, heads, 0, batch, heads, L,
+                          frames, audio_tokens, eps, (float*)out, st);
+  } else {
+    return fail(FH_ERR_ARG, "bad dtype");
+  }
+  if (e != cudaSuccess) return fail(FH_ERR_CUDA, "cross-attention launch: %s", cudaGetErrorString(e));
+  return FH_OK;
+}
+
+int fh_op_row_norm(const float* x, void* out, int M, int D, int mode, const float* a, const float* c, long bstride,
+                   int rows_per_batch, float eps, int dtype, void* stream) {
+  if (!x || !out || !a || !c || !aligned16(x) || !aligned16(out) || !aligned16(a) || !aligned16(c))
+    return fail(FH_ERR_ARG, "null or unaligned pointer");
+  if (M < 1 || rows_per_batch < 1 || mode < 0 || mode > 2 || bstride < 0)
+    return fail(FH_ERR_SHAPE, "bad row-norm arguments");
+  const int nv = D / 128;
+  if (D % 128 || !(nv == 1 || nv == 2 || nv == 3 || nv == 4 || nv == 6 || nv == 8 || nv == 12 || nv == 16))
+    return fail(FH_ERR_SHAPE, "row width %d not supported", D);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // norm_rows takes (shift, scale) for the modulated modes and (weight, bias) for mode 1
+  cudaError_t e;
+  if (dtype == FH_BF16)
+    e = mode == 1 ? norm_rows<bf16>(x, (bf16*)out, M, D, rows_per_batch, 1, nullptr, nullptr, 0, a, c, eps, st)
+                  : norm_rows<bf16>(x, (bf16*)out, M, D, rows_per_batch, mode, c, a, bstride, nullptr, nullptr, eps, st);
+  else if (dtype == FH_F32)
+    e = mode == 1 ? norm_rows<float>(x, (float*)out, M, D, rows_per_batch, 1, nullptr, nullptr, 0, a, c, eps, st)
+                  : norm_rows<float>(x, (float*)out, M, D, rows_per_batch, mode, c, a, bstride, nullptr, nullptr, eps,
+                                     st);
+  else
+    return fail(FH_ERR_ARG, "bad dtype");
+  if (e != cudaSuccess) return fail(FH_ERR_CUDA, "row-norm launch: %s", cudaGetErrorString(e));
   return FH_OK;
 }
 

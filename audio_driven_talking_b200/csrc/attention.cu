@@ -18,10 +18,11 @@
 //              its own running max and sum): the two halves are two independent
 //              partial attentions over disjoint key sets, combined once at the end with
 //              their maxima and sums (O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1)).
-//              P is written over the S columns it has consumed as two packed bf16 parts,
-//              P_hi = bf16(p) and P_lo = bf16(p - P_hi), both multiplied by V, so the
-//              weights enter the product with about 16 bits (bf16 P alone was the
-//              kernel's whole error: the split cuts its RMS error by a quarter). O_w stays
+//              P is written over the S columns it has consumed as packed fp16 (11-bit
+//              significand; p <= 2^8 by the rescale rule below) and multiplied by V, which
+//              the QKV epilogue stores in fp16 for this (a tensor-core product takes A and
+//              B of one type): the weights carry 8 times less rounding than bf16 P, which
+//              alone was the kernel's whole error, for one P.V product per key. O_w stays
 //              in TMEM; it is rescaled only when a row's running max grows by more than
 //              2^8 (then p <= 256 against the stale max, exact after the final division),
 //              so most tiles need no correction pass and the warpgroups never wait for
@@ -67,6 +68,37 @@ __device__ __forceinline__ float row_rms(const float* ssq, int ssq_ld, long row,
   float s = 0.f;
   for (int h = 0; h < heads; ++h) s += p[h];
   return rsqrtf(s * inv_d + eps);
+}
+
+// Every key's RMS factor rk[key] (0 past L) for keys [0, nkeys), by `nthreads` threads: with
+// 12 heads (the model's width) each row's 12 partial sums are three 16-byte loads, and a
+// thread issues the loads of its four rows before it adds any of them, so the prologue
+// costs about one round trip to L2 instead of one per row and head.
+__device__ __forceinline__ void key_rms_all(float* rk, const float* ssq, int ssq_ld, long row0, int heads, int L,
+                                            int nkeys, float inv_d, float eps, int t, int nthreads) {
+  if (heads == 12 && (ssq_ld & 3) == 0 && (reinterpret_cast<uintptr_t>(ssq) & 15) == 0) {
+    for (int base = 0; base < nkeys; base += 4 * nthreads) {
+      float4 v[4][3];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int key = base + u * nthreads + t;
+        const float4* p = reinterpret_cast<const float4*>(ssq + (row0 + (key < L ? key : 0)) * ssq_ld + heads);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) v[u][c] = p[c];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int key = base + u * nthreads + t;
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < 3; ++c) s += (v[u][c].x + v[u][c].y) + (v[u][c].z + v[u][c].w);
+        if (key < nkeys) rk[key] = key < L ? rsqrtf(s * inv_d + eps) : 0.f;
+      }
+    }
+  } else {
+    for (int key = t; key < nkeys; key += nthreads)
+      rk[key] = key < L ? row_rms(ssq, ssq_ld, row0 + key, heads, heads, inv_d, eps) : 0.f;
+  }
 }
 
 __global__ void __launch_bounds__(AT_THREADS, 1)
@@ -128,6 +160,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -192,7 +227,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id_s = idesc_bf16_f32(128, 128, false);
-      const uint32_t id_o = idesc_bf16_f32(128, 128, true);
+      const uint32_t id_o = idesc_f16_f32(128, 128, true);  // fp16 P (TMEM) and V (smem)
       const uint32_t q_addr = smem_u32(smem + OFF_Q);
       bool ok = mbar_wait(q_full, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       tc_fence_after();
@@ -229,10 +264,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
             }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              // keys 64w + 16(kk%4) .. +15: P_hi (kk < 4) in columns 64w + 8(kk%4), P_lo 32 further
-              const uint32_t a_tmem = tmem + bf * 128 + w * 64 + (kk >> 2) * 32 + (kk & 3) * 8;
-              const uint32_t b_off = (w * 64 + (kk & 3) * 16) * 128;  // 16 key rows of V
+            for (int kk = 0; kk < 4; ++kk) {
+              // keys 64w + 16kk .. +15: their P (fp16 pairs) in columns 64w + 8kk .. +7
+              const uint32_t a_tmem = tmem + bf * 128 + w * 64 + kk * 8;
+              const uint32_t b_off = (w * 64 + kk * 16) * 128;  // 16 key rows of V
               tc_mma_f16_ts(tmem + 256 + w * 128, a_tmem, sdesc_mnmajor_sw128(v_addr + b_off, PANEL), id_o,
                             (i > 0 || kk > 0) ? 1u : 0u);
             }
@@ -267,8 +302,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
 
     // every key's RMS factor, once per CTA (the keys are shared by all tiles of the row)
     float* rk_all = reinterpret_cast<float*>(smem + OFF_RKALL);
-    for (int key = t; key < nkv * AT_BK; key += AT_SOFTMAX_THREADS)
-      rk_all[key] = key < L ? row_rms(ssq, ssq_ld, (long)b * L + key, heads, heads, inv_d, eps) : 0.f;
+    key_rms_all(rk_all, ssq, ssq_ld, (long)b * L, heads, L, nkv * AT_BK, inv_d, eps, t, AT_SOFTMAX_THREADS);
     mbar_arrive(rk_full);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = mbar_wait(rk_full, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
@@ -341,11 +375,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         }
         m_run = m_new;
       }
-      // probabilities against the (possibly stale) running max, split into bf16 high and low
-      // parts; a row whose keys so far are all missing uses 0 as its reference (ex2(-inf) = 0)
+      // probabilities against the (possibly stale) running max, packed as fp16 pairs; a row
+      // whose keys so far are all missing uses 0 as its reference (ex2(-inf) = 0)
       const float mref = m_run == -INFINITY ? 0.f : m_run;
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pa[16], pb2[16], la[16], lb[16];
+      uint32_t pa[16], pb2[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const float p0 = ex2(fmaf(sa[2 * u], qscale, -mref));
@@ -353,21 +387,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
         const float q0 = ex2(fmaf(sb[2 * u], qscale, -mref));
         const float q1 = ex2(fmaf(sb[2 * u + 1], qscale, -mref));
         rs4[u & 3] += (p0 + p1) + (q0 + q1);
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(p0, p1);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(q0, q1);
-        const float2 f0 = __bfloat1622float2(h0), f1 = __bfloat1622float2(h1);
-        __nv_bfloat162 g0 = __floats2bfloat162_rn(p0 - f0.x, p1 - f0.y);
-        __nv_bfloat162 g1 = __floats2bfloat162_rn(q0 - f1.x, q1 - f1.y);
+        __half2 h0 = __floats2half2_rn(p0, p1);
+        __half2 h1 = __floats2half2_rn(q0, q1);
         pa[u] = *reinterpret_cast<uint32_t*>(&h0);
         pb2[u] = *reinterpret_cast<uint32_t*>(&h1);
-        la[u] = *reinterpret_cast<uint32_t*>(&g0);
-        lb[u] = *reinterpret_cast<uint32_t*>(&g1);
       }
       l_run += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      tmem_st16(s_t, pa);        // P_hi of keys 0..31 of this half -> columns 0..15 (already read)
-      tmem_st16(s_t + 16, pb2);  // P_hi of keys 32..63 -> columns 16..31
-      tmem_st16(s_t + 32, la);   // P_lo -> columns 32..63
-      tmem_st16(s_t + 48, lb);
+      tmem_st16(s_t, pa);        // P of keys 0..31 of this half -> columns 0..15 (already read)
+      tmem_st16(s_t + 16, pb2);  // P of keys 32..63 -> columns 16..31
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[2 * half + bf]);
@@ -412,6 +439,9 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
   }
 
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

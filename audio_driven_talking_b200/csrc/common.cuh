@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -132,6 +133,12 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 // Make generic-proxy shared-memory writes visible to the async proxy (tensor core reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Order this thread's global-memory accesses of the async proxy (TMA) with its generic ones:
+// after a bulk store has completed and before a flag publishes it, and after a flag has been
+// acquired and before a TMA load reads what it published.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // TMA store of a shared-memory box to global memory, and the same with an fp32 add at the
@@ -266,6 +273,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
   return (1u << 4)                       // D format: f32
          | (1u << 7)                     // A format: bf16
          | (1u << 10)                    // B format: bf16
+         | ((b_mn_major ? 1u : 0u) << 16)  // B major-ness
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor of kind::f16: fp16 A and B, fp32 D, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
+  return (1u << 4)                       // D format: f32
+         | (0u << 7)                     // A format: f16
+         | (0u << 10)                    // B format: f16
          | ((b_mn_major ? 1u : 0u) << 16)  // B major-ness
          | ((uint32_t)(N >> 3) << 17)    // N / 8
          | ((uint32_t)(M >> 4) << 24);   // M / 16
@@ -439,6 +456,12 @@ __device__ __forceinline__ void store8(bf16* dst, const float* v) {
   __nv_bfloat162 h[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(h);
+}
+__device__ __forceinline__ void store8(__half* dst, const float* v) {
+  __half2 h[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
   *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(h);
 }
 __device__ __forceinline__ void store8(float* dst, const float* v) {

@@ -12,7 +12,9 @@
 //              q and k: full-width RMSNorm split per head, reading R4)
 //   EPI_QKV    as EPI_NORM for the q and k sections, plus 3D rotary on adjacent
 //              pairs (2d, 2d+1) of q and k, and a head-major scatter of q, k, v to
-//              [3][B][heads][L][128] (reading R3).
+//              [3][B][heads][L][128] (reading R3). With bf16 outputs q and k are bf16
+//              and v is fp16 (11-bit significand): the attention kernel multiplies it by
+//              fp16 softmax weights P, and a tensor-core product takes A and B of one type.
 // The RMS factor r = (sum(ssq)/D + eps)^-1/2 itself is applied later, inside the
 // attention kernels, to the scores: r is one scalar per row and both the gain and
 // the rotation are linear per channel, so RoPE(g * r * y) = r * RoPE(g * y).
@@ -40,9 +42,28 @@ struct EpiParams {
   int ssq_ld;
   int norm_period;        // column c is normed iff (c % norm_period) < norm_count
   int norm_count;
-  const float2* rope;     // EPI_QKV: (cos, sin) [rows_per_batch, 64]
+  // EPI_QKV: the rotary (cos, sin) per axis: [F][pf] for the frame index, then [H][ph] for the
+  // row, then [W][pw] for the column (pf + ph + pw = 64 pairs); token l = (f H + r) W + c
+  const float2* rope;
+  int rope_H, rope_W, rope_pf, rope_ph, rope_off_h, rope_off_w;
   int dim;                // EPI_QKV: width D of each of the q, k, v sections
   long sec_stride;        // EPI_QKV: elements per section = B * heads * L * 128
+  // CTA-pair GEMM, stream-K: fp32 partial sums [clusters][2][128][BN] and per-(tile, CTA,
+  // 32-row quarter) counters (zero between launches); null sk_part: whole tiles per cluster
+  float* sk_part;
+  int* sk_flags;
+  // EPI_RESID on CTA pairs (width 1536): once every CTA of the launch has added its tiles to
+  // the residual, the CTAs normalise its rows for the next step (rownorm.cuh, mode ln_mode)
+  // into ln_out [M, N] bf16; ln_a / ln_c are the scale / shift (modes 0, 2; stride
+  // ln_bstride per stream) or weight / bias (mode 1) vectors; ln_ctr a counter, zero on entry,
+  // that no other launch uses. ln_out null: no norm.
+  void* ln_out;
+  int ln_mode;
+  const float* ln_a;
+  const float* ln_c;
+  long ln_bstride;
+  float ln_eps;
+  int* ln_ctr;
 };
 
 __device__ __forceinline__ bool epi_normed(const EpiParams& p, int col) {
@@ -96,14 +117,24 @@ __device__ __forceinline__ void epi_math(const EpiParams& p, int row, int col0, 
 }
 
 // EPI_QKV on q and k columns: rotate adjacent pairs (2d, 2d+1) by the angles of the row's
-// token position (table (cos, sin) [rows_per_batch, 64]).
+// token position. A pair turns with one axis only (reading R3), so its (cos, sin) comes from
+// that axis's small table (a few KB: it stays in L1 for every row of a tile).
 __device__ __forceinline__ void epi_rope(const EpiParams& p, int row, int col0, float (&v)[32]) {
   const int l = row % p.rows_per_batch;
-  const int d0 = (col0 % p.dim) & 127;
-  const float2* rt = p.rope + (long)l * 64 + (d0 >> 1);
+  const int hw = p.rope_H * p.rope_W;
+  const int f = l / hw, r = (l / p.rope_W) % p.rope_H, c = l % p.rope_W;
+  const int pf = p.rope_pf, pfh = p.rope_pf + p.rope_ph, pw = 64 - pfh;
+  const int pair0 = ((col0 % p.dim) & 127) >> 1;
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
-    float2 cs = rt[j >> 1];
+    const int d = pair0 + (j >> 1);  // the same for every lane
+    float2 cs;
+    if (d < pf)
+      cs = p.rope[f * pf + d];
+    else if (d < pfh)
+      cs = p.rope[p.rope_off_h + r * p.rope_ph + (d - pf)];
+    else
+      cs = p.rope[p.rope_off_w + c * pw + (d - pfh)];
     float x0 = v[j], x1 = v[j + 1];
     v[j] = x0 * cs.x - x1 * cs.y;
     v[j + 1] = x0 * cs.y + x1 * cs.x;
@@ -127,9 +158,9 @@ __device__ __forceinline__ void epi_prefetch(const EpiParams& p, int row, int co
       if (epi_normed(p, col0 + c)) prefetch_l1(p.gain + col0 + c);
     }
   }
-  if constexpr (KIND == EPI_QKV) {  // the row's rotary angles (64 (cos, sin) pairs, 4 lines)
-    const float2* rt = p.rope + (long)(row % p.rows_per_batch) * 64;
-    for (int c = 0; c < 64; c += 16) prefetch_l1(rt + c);
+  if constexpr (KIND == EPI_QKV) {  // the rotary tables (a few KB): one 128-byte line per lane
+    const int n = p.rope_off_w + p.rope_W * (64 - p.rope_pf - p.rope_ph);
+    for (int i = (threadIdx.x & 31) * 16; i < n; i += 32 * 16) prefetch_l1(p.rope + i);
   }
 }
 
@@ -168,8 +199,13 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, int row, int col0,
       const int heads = p.dim >> 7;
       OutT* dst = reinterpret_cast<OutT*>(p.out) + (long)sec * p.sec_stride +
                   (((long)bidx * heads + head) * p.rows_per_batch + l) * 128 + d0;
+      if (std::is_same<OutT, bf16>::value && sec == 2) {  // v in fp16 (see EPI_QKV above)
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) store8(dst + j, v + j);
+        for (int j = 0; j < 32; j += 8) store8(reinterpret_cast<__half*>(dst) + j, v + j);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) store8(dst + j, v + j);
+      }
     }
   }
 }
@@ -209,6 +245,11 @@ __device__ __forceinline__ void stage_row(uint8_t* box, int r, const float (&v)[
   uint8_t* row = box + r * 64;
 #pragma unroll
   for (int j = 0; j < 4; ++j) store8(reinterpret_cast<bf16*>(row + ((j ^ ((r >> 1) & 3)) << 4)), v + 8 * j);
+}
+__device__ __forceinline__ void stage_row(uint8_t* box, int r, const float (&v)[32], __half*) {
+  uint8_t* row = box + r * 64;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) store8(reinterpret_cast<__half*>(row + ((j ^ ((r >> 1) & 3)) << 4)), v + 8 * j);
 }
 
 template <int KIND>

@@ -5,7 +5,7 @@
 // contiguous). This is every dense contraction of the DiT: patch embed, QKV,
 // O-proj, cross-Q, cross-KV, cross-O, FFN1, FFN2 and the head.
 //
-// Three kernels, all warp-specialised with 192 threads:
+// Two kernels, both warp-specialised with 192 threads:
 //   warp 0     TMA producer: one thread streams 64-deep A and W tiles with the
 //              128-byte swizzle into a STAGES-deep shared-memory ring (per-CTA
 //              loads, no cluster multicast), the first stages' W before the
@@ -20,12 +20,12 @@
 //                   (cta_group::1), two accumulators so the epilogue of tile i
 //                   overlaps the MMAs of tile i+1, direct 16-byte stores.
 // gemm_tc2_kernel   a CTA pair (cluster of 2) per 256 x BN tile (cta_group::2),
-//                   persistent, two accumulators; the epilogue stages 32 x 32
-//                   boxes in shared memory and stores them by TMA (the residual
-//                   as a TMA fp32 reduce-add into x).
-// gemm_tc2s_kernel  split-K: one 256 x 256 tile per cluster of four CTAs (two
-//                   pairs, half of K each), reduce-scattered between the pairs
-//                   through shared memory, then the same staged epilogue.
+//                   persistent over a stream-K share of the tiles' k-blocks (one
+//                   cluster per CTA pair of the GPU, every share the same size;
+//                   tiles cut between clusters are summed by the owner through
+//                   fp32 partials in the workspace), two accumulators; the
+//                   epilogue stages 32 x 32 boxes in shared memory and stores them
+//                   by TMA (the residual as a TMA fp32 reduce-add into x).
 // Every wait is bounded (FH_WAIT_LIMIT_NS); on expiry the CTA latches an error
 // bit, lets the producer's in-flight copies land, frees TMEM and exits.
 #include <cstdio>
@@ -33,6 +33,7 @@
 
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "rownorm.cuh"
 
 namespace fh {
 
@@ -40,6 +41,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
+constexpr int SK_COLS = 256;  // columns of a stream-K partial-sum slot row (the widest tile)
 
 template <int BN>
 struct TcShape {
@@ -89,6 +91,9 @@ __global__ void __launch_bounds__(192, 1)
     tmem_alloc(tmem_holder, 2 * BN);
     tmem_relinquish();
   }
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -253,6 +258,9 @@ __global__ void __launch_bounds__(192, 1)
     }
   }
 
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -277,6 +285,21 @@ cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, int M, int N, 
 // M=256 MMAs that read both CTAs' shared memory, and each CTA's TMEM receives its 128
 // rows. Per unit of MMA work a CTA streams A + W/2 instead of A + W, which is what the
 // per-SM operand bandwidth limits at these sizes. All loads are per-CTA (no multicast).
+//
+// Work split (stream-K): the tiles' 64-deep k-blocks, taken tile by tile (tiles in
+// m-fastest order, so clusters working at the same time share W n-tiles in L2), form one
+// range of units that is cut into equal contiguous shares, one per cluster. A cluster's
+// share is a sequence of segments (tile, k-blocks [kb0, kb1)). A segment that covers a
+// whole tile runs the epilogue. Where a tile is cut between clusters, the segment that
+// starts at k-block 0 is its owner and the later ones are contributors: a contributor is
+// always the first segment of its cluster's share and the owner the last of its own, so
+// contributors finish early and no cluster waits on one that is waiting itself. A
+// contributor stores its fp32 partial accumulator in its cluster's slot of the workspace
+// (`sk_part`) and counts itself on the tile's flag; the owner waits for the count, adds
+// the contributors' partials in k order (a fixed order: the result is deterministic),
+// runs the epilogue and clears the flag for the next launch (flags are per 32-row quarter
+// of a CTA's rows, so each epilogue warp waits only for the same rows). Without a partial buffer
+// (`sk_part` null) the shares are whole tiles.
 template <int BN>
 struct Tc2Shape {
   static constexpr int BNH = BN / 2;
@@ -290,17 +313,65 @@ struct Tc2Shape {
   static constexpr uint32_t RING_BYTES = STAGES * STAGE_BYTES;
   // epilogue staging: per epilogue warp two 32-row boxes of up to 128-byte rows
   static constexpr uint32_t STG_BYTES = 4 * 2 * 4096;
-  static constexpr uint32_t SMEM = RING_BYTES + STG_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+  // a stream-K owner's epilogue warps receive the contributors' partial sums as 32 x 32 fp32
+  // boxes in the operand ring (idle by then): PBOX boxes per warp, loaded ahead by TMA
+  static constexpr int PBOX = RING_BYTES / (4 * 4096) < 12 ? RING_BYTES / (4 * 4096) : 12;
+  static constexpr uint32_t SMEM = RING_BYTES + STG_BYTES + 1024 /*align*/ + 1024 /*barriers*/;
 };
+
+// One segment of a cluster's work: k-blocks [kb0, kb1) of one tile.
+struct SkSeg {
+  int tile, kb0, kb1;
+};
+// A cluster's segments. Stream-K (sk): the k-blocks of all tiles, tile by tile, form one range
+// of units cut into equal contiguous shares, one per cluster. Whole tiles (!sk): cluster c takes
+// tiles c, c + ncl, c + 2 ncl, ... (so the clusters working at the same time cover consecutive
+// tiles, which share W n-tiles in L2).
+struct SkRange {
+  long total;  // stream-K units: k-blocks of all tiles
+  int nk, ncl, ntiles;
+  bool sk;
+  __device__ __forceinline__ long lo(int c) const { return (long)c * total / ncl; }
+  // the first position of cluster c's work, and whether position u is still inside it
+  __device__ __forceinline__ long begin(int c) const { return sk ? lo(c) : c; }
+  __device__ __forceinline__ bool more(int c, long u) const { return sk ? u < lo(c + 1) : u < ntiles; }
+  // the segment at position u of cluster c's work; returns the next position
+  __device__ __forceinline__ long seg(int c, long u, SkSeg& s) const {
+    if (!sk) {
+      s.tile = (int)u;
+      s.kb0 = 0;
+      s.kb1 = nk;
+      return u + ncl;
+    }
+    const long uh = lo(c + 1);
+    s.tile = (int)(u / nk);
+    s.kb0 = (int)(u - (long)s.tile * nk);
+    const long rem = uh - u;
+    s.kb1 = (long)(nk - s.kb0) <= rem ? nk : s.kb0 + (int)rem;
+    return u + (s.kb1 - s.kb0);
+  }
+  // clusters after `cl` whose shares hold later k-blocks of `tile` (its contributors)
+  __device__ __forceinline__ int contributors(int tile, int cl) const {
+    const long end = (long)(tile + 1) * nk;
+    int n = 0;
+    for (int c = cl + 1; c < ncl && lo(c) < end; ++c) ++n;
+    return n;
+  }
+};
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
 template <int BN, int KIND, typename OutT>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep, unsigned* err) {
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmP, int M, int N,
+                    int K, EpiParams ep, unsigned* err) {
   using S = Tc2Shape<BN>;
-  // every epilogue leaves through shared memory and TMA stores (EPI_QKV: a 3D map over the
-  // head-major [3 * B * heads][L][128] layout, except for warps whose rows cross a stream)
-  constexpr bool STAGED = true;
+  static_assert(BN <= SK_COLS, "a partial-sum slot row holds SK_COLS columns");
   // element type of the staged boxes: the fp32 residual for EPI_RESID, else the output type
   using StageT = typename std::conditional<KIND == EPI_RESID, float, OutT>::type;
   extern __shared__ uint8_t smem_raw[];
@@ -310,17 +381,25 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = empty + S::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* dealloc_bar = tempty + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(dealloc_bar + 1);
+  uint64_t* pbar = dealloc_bar + 1;  // [4 warps][PBOX] partial-sum boxes landed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(pbar + 4 * S::PBOX);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();  // 0: the CTA that issues the pair's MMAs
-  const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const int cl = blockIdx.x >> 1;
   const int num_m = (M + 2 * BM - 1) / (2 * BM);
   const int num_n = N / BN;
   const int ntiles = num_m * num_n;
   const int nk = (K + BK - 1) / BK;
+  SkRange R;
+  R.sk = ep.sk_part != nullptr;
+  R.nk = nk;
+  R.ncl = gridDim.x >> 1;
+  R.ntiles = ntiles;
+  R.total = (long)ntiles * nk;
+  const long u_begin = R.begin(cl);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
@@ -332,11 +411,13 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&tempty[a], 2 * 128);  // both CTAs' epilogue threads
     }
     mbar_init(dealloc_bar, 1);
+    for (int i = 0; i < 4 * S::PBOX; ++i) mbar_init(&pbar[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
-    if (STAGED) prefetch_tmap(&tmC);
+    prefetch_tmap(&tmC);
+    if (R.sk) prefetch_tmap(&tmP);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_holder, S::TMEM_COLS);
@@ -350,15 +431,18 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {
       // The weights W are never written by any kernel: stream the first stages' W halves
-      // before waiting for the kernels this one depends on (programmatic launch).
+      // of the share's first segment before waiting for the kernels this one depends on
+      // (programmatic launch).
       int pre = 0;
-      if (cl < ntiles) {
-        const int n0 = (cl / num_m) * BN + (int)rank * S::BNH;
-        pre = nk < S::STAGES ? nk : S::STAGES;
+      if (R.more(cl, u_begin)) {
+        SkSeg s0;
+        R.seg(cl, u_begin, s0);
+        const int n0 = (s0.tile / num_m) * BN + (int)rank * S::BNH;
+        pre = s0.kb1 - s0.kb0 < S::STAGES ? s0.kb1 - s0.kb0 : S::STAGES;
         for (int s = 0; s < pre; ++s) {
           if (rank == 0) mbar_expect_tx(&full[s], S::TX_BYTES);
-          tma_load_2d_pair(&tmB, mapa_shared(smem_u32(&full[s]), 0), smem + s * S::STAGE_BYTES + S::A_BYTES, s * BK,
-                           n0);
+          tma_load_2d_pair(&tmB, mapa_shared(smem_u32(&full[s]), 0), smem + s * S::STAGE_BYTES + S::A_BYTES,
+                           (s0.kb0 + s) * BK, n0);
         }
       }
       pdl_wait();
@@ -366,14 +450,16 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0;
       int issues = 0;
       bool first = true;
-      for (int tile = cl; tile < ntiles; tile += ncl, first = false) {
-        const int m0 = (tile % num_m) * 2 * BM + (int)rank * BM;
-        const int n0 = (tile / num_m) * BN + (int)rank * S::BNH;
-        for (int kb = 0; kb < nk; ++kb) {
+      for (long u = u_begin; R.more(cl, u); first = false) {
+        SkSeg sg;
+        u = R.seg(cl, u, sg);
+        const int m0 = (sg.tile % num_m) * 2 * BM + (int)rank * BM;
+        const int n0 = (sg.tile / num_m) * BN + (int)rank * S::BNH;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) goto producer_done;
           uint8_t* sa = smem + stage * S::STAGE_BYTES;
           const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
-          if (!(first && kb < pre)) {
+          if (!(first && kb - sg.kb0 < pre)) {
             if (rank == 0) mbar_expect_tx(&full[stage], S::TX_BYTES);
             tma_load_2d_pair(&tmB, bar0, sa + S::A_BYTES, kb * BK, n0);
           }
@@ -412,14 +498,16 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
-      for (int tile = cl; tile < ntiles; tile += ncl, ++local) {
+      for (long u = u_begin; R.more(cl, u); ++local) {
+        SkSeg sg;
+        u = R.seg(cl, u, sg);
         const int acc = local & 1;
         const uint32_t aph = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, err, ERRBIT_TIMEOUT_GEMM)) {
             ok = false;
             break;
@@ -430,7 +518,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             tc_mma_f16_pair(d_tmem, sdesc_kmajor_sw128(a_addr + k * 32), sdesc_kmajor_sw128(b_addr + k * 32), idesc,
-                            (kb | k) != 0 ? 1u : 0u);
+                            (kb > sg.kb0 || k > 0) ? 1u : 0u);
           }
           tc_commit_pair(&empty[stage], 0x3);
           if (++stage == S::STAGES) {
@@ -454,100 +542,195 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t nchunk = 0;
     pdl_wait();
     int local = 0;
-    for (int tile = cl; tile < ntiles; tile += ncl, ++local) {
+    for (long u = u_begin; R.more(cl, u); ++local) {
+      SkSeg sg;
+      u = R.seg(cl, u, sg);
       const int acc = local & 1;
       const uint32_t aph = (local >> 1) & 1;
-      const int m0 = (tile % num_m) * 2 * BM + (int)rank * BM;
-      const int n0 = (tile / num_m) * BN;
+      const int m0 = (sg.tile % num_m) * 2 * BM + (int)rank * BM;
+      const int n0 = (sg.tile / num_m) * BN;
       const int row = m0 + quarter * 32 + lane;
+      const int row0 = m0 + quarter * 32;
       const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      if constexpr (STAGED) {
-        // 32 x 32 boxes: this warp's 32 rows, 32 columns at a time, through two staging
-        // buffers; lane 0 issues the TMA store (the residual: an fp32 add in L2)
-        const int row0 = m0 + quarter * 32;
-        epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0, BN);  // while the MMAs run
+      // one flag per (tile, CTA of the pair, 32-row quarter): the owner's warp for these rows
+      // waits only for the contributors' warps that stored the same rows
+      int* flag = R.sk ? ep.sk_flags + (2 * sg.tile + (int)rank) * 4 + quarter : nullptr;
+      if (sg.kb0 > 0) {
+        // contributor: each thread stores its row's raw fp32 partial sums straight from the
+        // accumulator into this cluster's slot (row-major rows of SK_COLS floats, which the
+        // owner reads back as 32 x 32 TMA boxes); once the warp's stores are visible the
+        // quarter's flag counts them
         bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
         if (!__all_sync(0xffffffffu, ok)) break;
         tc_fence_after();
-        // EPI_QKV: the 32 rows stay inside one stream (row0 and L both multiples of 32 at
-        // the usual sizes); otherwise this warp stores directly, row by row
-        bool direct = false;
-        int l0 = 0, bidx = 0;
-        if constexpr (KIND == EPI_QKV) {
-          l0 = row0 % ep.rows_per_batch;
-          bidx = row0 / ep.rows_per_batch;
-          direct = l0 + 32 > ep.rows_per_batch && row0 + (ep.rows_per_batch - l0) < M;
-        }
+        float* prow = ep.sk_part + ((size_t)(cl * 2 + (int)rank) * BM + quarter * 32 + lane) * SK_COLS;
 #pragma unroll 1
-        for (int g = 0; row0 < M && g < BN; g += 128) {  // a warp with no row below M stores nothing
-          float ssq = 0.f;
-#pragma unroll 1
-          for (int c = 0; c < 128 && g + c < BN; c += 32) {
-            float v[32];
-            tmem_ld32(tb + g + c, v);
-            tc_wait_ld();
-            if (direct) {
-              if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
-              continue;
-            }
-            if (row < M) {
-              epi_math<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
-              if constexpr (KIND == EPI_QKV)
-                if (epi_normed(ep, n0 + g + c)) epi_rope(ep, row, n0 + g + c, v);
-            } else {
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          tmem_ld32(tb + c, v);
+          tc_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = 0.f;
-            }
-            // buffers alternate per committed store, so the one group that may still be
-            // reading is the other buffer's
-            uint8_t* box = stg + (nchunk & 1) * 4096;
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
+          for (int j = 0; j < 8; ++j)
+            __stcg(reinterpret_cast<float4*>(prow + c + 4 * j), make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]));
+        }
+        tc_fence_before();
+        mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();  // the warp's partial sums are visible before the flag counts them
+          atomicAdd(flag, 1);
+        }
+        __syncwarp();
+        continue;
+      }
+      // whole tile, or the owner of a cut tile: wait for its contributors' partial sums
+      const int ncontrib = (R.sk && sg.kb1 < nk) ? R.contributors(sg.tile, cl) : 0;
+      epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0, BN);  // while the MMAs run
+      bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
+      if (ncontrib > 0 && lane == 0 && ok) {
+        const uint64_t t0 = globaltimer();
+        while (ld_acquire(flag) < ncontrib) {
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          if (globaltimer() - t0 > FH_WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            if (err) atomicOr(err, ERRBIT_TIMEOUT_GEMM);
+            ok = false;
+            break;
+          }
+        }
+        fence_proxy_async_global();
+      }
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      // the contributors' boxes (32 rows x 32 columns each, box i = chunk * ncontrib + q) stream
+      // into this warp's PBOX buffers in the ring (free: this owner segment is the share's last,
+      // its MMAs are done), up to PBOX ahead of their use
+      uint8_t* pbuf = smem + quarter * (S::PBOX * 4096);
+      uint64_t* pb = pbar + quarter * S::PBOX;
+      const int nbox = ncontrib * (BN / 32);
+      auto issue_box = [&](int i) {
+        const int q = i % ncontrib, ch = i / ncontrib;
+        const int slot = i % S::PBOX;
+        mbar_expect_tx(&pb[slot], 4096);
+        tma_load_2d(&tmP, &pb[slot], pbuf + slot * 4096, ch * 32, ((cl + 1 + q) * 2 + (int)rank) * BM + quarter * 32);
+      };
+      int nissued = 0;  // boxes issued (lane 0) and waited for
+      if (lane == 0)
+        for (; nissued < nbox && nissued < S::PBOX; ++nissued) issue_box(nissued);
+      int nwait = 0;
+      bool pok = true;  // every box arrived in time
+      // EPI_QKV: the 32 rows stay inside one stream (row0 and L both multiples of 32 at
+      // the usual sizes); otherwise this warp stores directly, row by row
+      bool direct = false;
+      int l0 = 0, bidx = 0;
+      if constexpr (KIND == EPI_QKV) {
+        l0 = row0 % ep.rows_per_batch;
+        bidx = row0 / ep.rows_per_batch;
+        direct = l0 + 32 > ep.rows_per_batch && row0 + (ep.rows_per_batch - l0) < M;
+      }
+      // one 32-column chunk of the tile: contributors' partial sums, the epilogue, the store
+      float ssq = 0.f;
+      auto chunk = [&](float (&v)[32], int c) {
+        // contributors' partial sums of these 32 columns, in k order
+        for (int q = 0; q < ncontrib && pok; ++q, ++nwait) {
+          const int slot = nwait % S::PBOX;
+          pok = __all_sync(0xffffffffu,
+                           mbar_wait(&pb[slot], (nwait / S::PBOX) & 1, abort_flag, err, ERRBIT_TIMEOUT_GEMM));
+          if (!pok) break;
+          const uint8_t* prow = pbuf + slot * 4096 + lane * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 pp = *reinterpret_cast<const float4*>(prow + ((j ^ (lane & 7)) << 4));
+            v[4 * j] += pp.x;
+            v[4 * j + 1] += pp.y;
+            v[4 * j + 2] += pp.z;
+            v[4 * j + 3] += pp.w;
+          }
+          __syncwarp();
+          if (lane == 0 && nissued < nbox) issue_box(nissued++);  // its buffer has been read
+        }
+        if (row0 >= M) return;  // a warp with no row below M stores nothing
+        if (direct) {
+          if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + c, v, ssq);
+        } else {
+          if (row < M) {
+            epi_math<KIND, OutT>(ep, row, n0 + c, v, ssq);
+            if constexpr (KIND == EPI_QKV)
+              if (epi_normed(ep, n0 + c)) epi_rope(ep, row, n0 + c, v);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = 0.f;
+          }
+          // buffers alternate per committed store, so the one group that may still be
+          // reading is the other buffer's
+          uint8_t* box = stg + (nchunk & 1) * 4096;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          if (KIND == EPI_QKV && std::is_same<OutT, bf16>::value && (n0 + c) / ep.dim == 2)
+            stage_row(box, lane, v, (__half*)nullptr);  // v in fp16 (epilogue.cuh, EPI_QKV)
+          else
             stage_row(box, lane, v, (StageT*)nullptr);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              const int col = n0 + g + c;
-              if constexpr (KIND == EPI_RESID) {
-                tma_reduce_add_2d(&tmC, box, col, row0);  // rows at or past M are clipped
-              } else if constexpr (KIND == EPI_QKV) {
-                const int sec = col / ep.dim, cin = col - sec * ep.dim;
-                const int heads = ep.dim >> 7;
-                const int nb = M / ep.rows_per_batch;
-                tma_store_3d(&tmC, box, cin & 127, l0, (sec * nb + bidx) * heads + (cin >> 7));
-              } else {
-                tma_store_2d(&tmC, box, col, row0);
-              }
-              bulk_commit();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int col = n0 + c;
+            if constexpr (KIND == EPI_RESID) {
+              tma_reduce_add_2d(&tmC, box, col, row0);  // rows at or past M are clipped
+            } else if constexpr (KIND == EPI_QKV) {
+              const int sec = col / ep.dim, cin = col - sec * ep.dim;
+              const int heads = ep.dim >> 7;
+              const int nb = M / ep.rows_per_batch;
+              tma_store_3d(&tmC, box, cin & 127, l0, (sec * nb + bidx) * heads + (cin >> 7));
+            } else {
+              tma_store_2d(&tmC, box, col, row0);
             }
-            ++nchunk;
+            bulk_commit();
           }
-          if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
+          ++nchunk;
         }
-      } else {
-        bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int g = 0; g < BN; g += 128) {
-          float ssq = 0.f;
-#pragma unroll 1
-          for (int c = 0; c < 128 && g + c < BN; c += 32) {
-            float v[32];
-            tmem_ld32(tb + g + c, v);
-            tc_wait_ld();
-            if (row < M) epi_chunk<KIND, OutT>(ep, row, n0 + g + c, v, ssq);
-          }
-          if (row < M) epi_group_end<KIND>(ep, row, n0 + g, ssq);
+        if ((c & 127) == 96 || c + 32 == BN) {  // the end of a 128-column group
+          if (row < M) epi_group_end<KIND>(ep, row, n0 + (c & ~127), ssq);
+          ssq = 0.f;
         }
+      };
+      // the accumulator's chunks leave TMEM one ahead of their use: each wait covers the
+      // chunk loaded while the previous one was being processed
+      float va[32], vb[32];
+      tmem_ld32(tb, va);
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 64) {
+        tc_wait_ld();
+        if (c + 32 < BN) tmem_ld32(tb + c + 32, vb);
+        chunk(va, c);
+        if (c + 32 >= BN) break;
+        tc_wait_ld();
+        if (c + 64 < BN) tmem_ld32(tb + c + 64, va);
+        chunk(vb, c + 32);
+      }
+      if (!pok) {
+        // boxes still in flight land before the CTA's shared memory can go away
+        if (lane == 0)
+          for (int i = nwait; i < nissued; ++i) drain_wait(&pb[i % S::PBOX], (i / S::PBOX) & 1);
+        __syncwarp();
+        break;
       }
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      if (ncontrib > 0 && lane == 0) *flag = 0;  // its only reader is done: clear it for the next launch
     }
-    if (STAGED && lane == 0) bulk_wait_all();  // every store issued by this warp has been performed
+    if (lane == 0) {
+      bulk_wait_all();  // every store issued by this warp has been performed
+      if (KIND == EPI_RESID && ep.ln_out) fence_proxy_async_global();  // ... before the rows are read back
+    }
     __syncwarp();
   }
 
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -560,15 +743,62 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
   }
+  if constexpr (KIND == EPI_RESID) {
+    if (ep.ln_out && N == 12 * 128) {
+      // the next norm of the updated rows: wait until every CTA of the launch (all resident:
+      // one cluster per CTA pair that fits) has added its tiles, then each warp normalises rows
+      if (threadIdx.x == 0 && !*abort_flag) {
+        __threadfence();
+        atomicAdd(ep.ln_ctr, 1);
+        const uint64_t t0 = globaltimer();
+        while (ld_acquire(ep.ln_ctr) < (int)gridDim.x) {
+          if (globaltimer() - t0 > FH_WAIT_LIMIT_NS) {
+            *abort_flag = 1;
+            if (err) atomicOr(err, ERRBIT_TIMEOUT_GEMM);
+            break;
+          }
+        }
+        __threadfence();
+      }
+      __syncwarp();  // warp 0 converged again before the CTA barrier
+      __syncthreads();
+      if (!*abort_flag) {
+        const int nw = blockDim.x >> 5;
+        for (int r = blockIdx.x * nw + warp; r < M; r += gridDim.x * nw) {
+          const long mb = (long)(r / ep.rows_per_batch) * ep.ln_bstride;
+          norm_row<bf16, 12>(ep.resid + (long)r * ep.ldr, reinterpret_cast<bf16*>(ep.ln_out) + (long)r * N, lane,
+                             ep.ln_mode, ep.ln_a + mb, ep.ln_c + mb, ep.ln_eps);
+        }
+      }
+    }
+  }
+}
+
+// CTA pairs of the pair GEMM, and clusters of four of the split-K kernel, that can be
+// resident at once, per device (set by gemm_tc_prepare): a stream-K owner waits for
+// contributors with higher cluster indices, and a split-K cluster's pairs wait for each
+// other, so every cluster of a launch must be able to run at the same time.
+int g_pair_clusters[64] = {0};
+int g_split_clusters[64] = {0};
+
+// Clusters of a pair-GEMM launch: one per CTA pair that can be resident, or fewer when there
+// is less work than that (stream-K: fewer k-blocks; whole tiles: fewer tiles).
+inline int tc2_clusters(int M, int N, int K, int bn, int num_sms, bool sk) {
+  const long tiles = (long)((M + 2 * BM - 1) / (2 * BM)) * (N / bn);
+  const long units = sk ? tiles * ((K + BK - 1) / BK) : tiles;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int cap = num_sms / 2;
+  const int resident = dev >= 0 && dev < 64 ? g_pair_clusters[dev] : 0;
+  if (resident > 0 && resident < cap) cap = resident;
+  return units < cap ? (int)units : cap;
 }
 
 template <int BN, int KIND, typename OutT>
-cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, int M, int N, int K,
-                       const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st) {
+cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, const CUtensorMap& p, int M,
+                       int N, int K, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st) {
   using S = Tc2Shape<BN>;
-  const int tiles = ((M + 2 * BM - 1) / (2 * BM)) * (N / BN);
-  int clusters = num_sms / 2;
-  if (tiles < clusters) clusters = tiles;
+  const int clusters = tc2_clusters(M, N, K, BN, num_sms, ep.sk_part != nullptr);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters);
   cfg.blockDim = dim3(192);
@@ -583,13 +813,7 @@ cudaError_t launch_tc2(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, KIND, OutT>, a, b, c, M, N, K, ep, err);
-}
-
-template <int BN, int KIND, typename OutT>
-cudaError_t prepare_tc2() {
-  return cudaFuncSetAttribute(gemm_tc2_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)Tc2Shape<BN>::SMEM);
+  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, KIND, OutT>, a, b, c, p, M, N, K, ep, err);
 }
 
 // ------------------------------------------------------------------ split-K over two CTA pairs
@@ -760,16 +984,24 @@ __global__ void __launch_bounds__(192, 1)
     epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0 + mine, HALF_COLS);
     if (ok && row0 < M) {
       uint8_t* out = smem + quarter * QBYTES;
-#pragma unroll 1
-      for (int c = 0; c < (int)HALF_COLS; c += 32) {
-        float v[32];
-        tmem_ld32(tb + theirs + c, v);
-        tc_wait_ld();
+      auto put = [&](const float (&v)[32], int c) {
         uint8_t* prow = out + (c >> 5) * 4096 + lane * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           *reinterpret_cast<float4*>(prow + ((j ^ (lane & 7)) << 4)) =
               make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      };
+      // chunks leave TMEM one ahead of their use (HALF_COLS is a multiple of 64)
+      float va[32], vb[32];
+      tmem_ld32(tb + theirs, va);
+#pragma unroll 1
+      for (int c = 0; c < (int)HALF_COLS; c += 64) {
+        tc_wait_ld();
+        tmem_ld32(tb + theirs + c + 32, vb);
+        put(va, c);
+        tc_wait_ld();
+        if (c + 64 < (int)HALF_COLS) tmem_ld32(tb + theirs + c + 64, va);
+        put(vb, c + 32);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -786,12 +1018,8 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t nchunk = 0;
     if (ok && row0 < M) {
       float ssq = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < (int)HALF_COLS; c += 32) {
+      auto chunk = [&](float (&v)[32], int c) {
         const int col = n0 + mine + c;
-        float v[32];
-        tmem_ld32(tb + mine + c, v);
-        tc_wait_ld();
         const uint8_t* prow = part + (c >> 5) * 4096 + lane * 128;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -821,6 +1049,18 @@ __global__ void __launch_bounds__(192, 1)
           bulk_commit();
         }
         ++nchunk;
+      };
+      // chunks leave TMEM one ahead of their use
+      float va[32], vb[32];
+      tmem_ld32(tb + mine, va);
+#pragma unroll 1
+      for (int c = 0; c < (int)HALF_COLS; c += 64) {
+        tc_wait_ld();
+        tmem_ld32(tb + mine + c + 32, vb);
+        chunk(va, c);
+        tc_wait_ld();
+        if (c + 64 < (int)HALF_COLS) tmem_ld32(tb + mine + c + 64, va);
+        chunk(vb, c + 32);
       }
       if (row < M) epi_group_end<KIND>(ep, row, n0 + mine, ssq);
     }
@@ -828,6 +1068,9 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   }
 
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -873,21 +1116,18 @@ cudaError_t prepare_tc2s() {
 }
 
 template <int BN, int KIND, typename OutT>
+cudaError_t prepare_tc2() {
+  return cudaFuncSetAttribute(gemm_tc2_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)Tc2Shape<BN>::SMEM);
+}
+
+template <int BN, int KIND, typename OutT>
 cudaError_t prepare_tc() {
   return cudaFuncSetAttribute(gemm_tc_kernel<BN, KIND, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)TcShape<BN>::SMEM);
 }
 
 }  // namespace
-
-// clusters of four of the split-K kernel that can be resident at once, per device
-int g_split_clusters[64] = {0};
-
-int current_device() {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  return dev;
-}
 
 cudaError_t gemm_tc_prepare() {
   const cudaError_t es[] = {
@@ -898,42 +1138,60 @@ cudaError_t gemm_tc_prepare() {
       prepare_tc2<128, EPI_STORE, bf16>(), prepare_tc2<256, EPI_STORE, bf16>(), prepare_tc2<128, EPI_GELU, bf16>(),
       prepare_tc2<256, EPI_GELU, bf16>(), prepare_tc2<128, EPI_NORM, bf16>(), prepare_tc2<256, EPI_NORM, bf16>(),
       prepare_tc2<128, EPI_QKV, bf16>(), prepare_tc2<256, EPI_QKV, bf16>(), prepare_tc2<128, EPI_RESID, bf16>(),
-      prepare_tc2<256, EPI_RESID, bf16>(), prepare_tc2<128, EPI_STORE, float>(),
-      prepare_tc2<256, EPI_STORE, float>(), prepare_tc2<224, EPI_GELU, bf16>(), prepare_tc2<224, EPI_STORE, float>(), prepare_tc2s<256, EPI_STORE, bf16>(), prepare_tc2s<256, EPI_NORM, bf16>(),
-      prepare_tc2s<256, EPI_RESID, bf16>(), prepare_tc2s<256, EPI_STORE, float>()};
+      prepare_tc2<256, EPI_RESID, bf16>(), prepare_tc2<128, EPI_STORE, float>(), prepare_tc2<256, EPI_STORE, float>(),
+      prepare_tc2<224, EPI_GELU, bf16>(), prepare_tc2<224, EPI_STORE, float>()};
   for (cudaError_t e : es)
     if (e != cudaSuccess) return e;
+  const cudaError_t es2[] = {prepare_tc2s<256, EPI_STORE, bf16>(), prepare_tc2s<256, EPI_NORM, bf16>(),
+                             prepare_tc2s<256, EPI_RESID, bf16>(), prepare_tc2s<256, EPI_STORE, float>()};
+  for (cudaError_t e : es2)
+    if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(4 * 64);
+  cfg.gridDim = dim3(2 * 64);
   cfg.blockDim = dim3(192);
   cfg.dynamicSmemBytes = Tc2Shape<256>::SMEM;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 4;
+  attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_tc2s_kernel<256, EPI_RESID, bf16>, &cfg);
+  cudaError_t e = cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<256, EPI_RESID, bf16>, &cfg);
   if (e != cudaSuccess) return e;
-  const int dev = current_device();
-  if (dev >= 0 && dev < 64) g_split_clusters[dev] = n;
+  int n4 = 0;
+  attr[0].val.clusterDim.x = 4;
+  cfg.gridDim = dim3(4 * 64);
+  e = cudaOccupancyMaxActiveClusters(&n4, gemm_tc2s_kernel<256, EPI_RESID, bf16>, &cfg);
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (n < 1) return cudaErrorInvalidConfiguration;
+  if (dev >= 0 && dev < 64) {
+    g_pair_clusters[dev] = n;
+    g_split_clusters[dev] = n4;
+  }
   return cudaSuccess;
 }
 
-cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, int M, int N, int K, int bn,
-                    int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
-                    bool pair) {
-  // the CTA-pair kernels store their epilogue through the output map `c`
+cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, const CUtensorMap* p, int M,
+                    int N, int K, int bn, int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms,
+                    cudaStream_t st, bool pair) {
+  // the CTA-pair kernels store their epilogue through the output map `c`, and stream-K moves
+  // partial sums through `p`
   if (pair && !c) return cudaErrorInvalidValue;
+  if (pair && ep.sk_part && (!p || !ep.sk_flags)) return cudaErrorInvalidValue;
   const CUtensorMap& cm = c ? *c : a;
-  // few 256 x 256 tiles (one per cluster of four fits the GPU): split K over two CTA pairs
+  const CUtensorMap& pm = p ? *p : cm;
+  // few 256 x 256 tiles (one per cluster of four fits the GPU), whole tiles asked for: split K
+  // over two CTA pairs of a cluster
   const int tiles256 = ((M + 2 * BM - 1) / (2 * BM)) * (N / 256);
-  const int dev = current_device();
-  const int resident = dev >= 0 && dev < 64 ? g_split_clusters[dev] : 0;
-  if (pair && bn == 256 && N <= 4096 && 4 * tiles256 <= num_sms && tiles256 <= resident && K >= 2 * BK &&
-      (kind == EPI_STORE || kind == EPI_NORM || kind == EPI_RESID)) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int resident4 = dev >= 0 && dev < 64 ? g_split_clusters[dev] : 0;
+  if (pair && !ep.sk_part && !ep.ln_out && bn == 256 && N <= 4096 && 4 * tiles256 <= num_sms &&
+      tiles256 <= resident4 && K >= 2 * BK && (kind == EPI_STORE || kind == EPI_NORM || kind == EPI_RESID)) {
     if (out_bf16) {
       if (kind == EPI_STORE) return launch_tc2s<256, EPI_STORE, bf16>(a, b, cm, M, N, K, ep, err, st);
       if (kind == EPI_NORM) return launch_tc2s<256, EPI_NORM, bf16>(a, b, cm, M, N, K, ep, err, st);
@@ -943,12 +1201,13 @@ cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
   }
 #define FH_TC_CASE(BNV, KV, OT)                                                                     \
   if (bn == BNV && kind == KV)                                                                      \
-    return pair ? launch_tc2<BNV, KV, OT>(a, b, cm, M, N, K, ep, err, num_sms, st)                  \
+    return pair ? launch_tc2<BNV, KV, OT>(a, b, cm, pm, M, N, K, ep, err, num_sms, st)              \
                 : launch_tc<BNV, KV, OT>(a, b, M, N, K, ep, err, num_sms, st);
   if (pair && bn == 224) {  // FFN1-shaped (8960 = 40 x 224 balances the waves)
-    if (kind == EPI_GELU && out_bf16) return launch_tc2<224, EPI_GELU, bf16>(a, b, cm, M, N, K, ep, err, num_sms, st);
+    if (kind == EPI_GELU && out_bf16)
+      return launch_tc2<224, EPI_GELU, bf16>(a, b, cm, pm, M, N, K, ep, err, num_sms, st);
     if (kind == EPI_STORE && !out_bf16)
-      return launch_tc2<224, EPI_STORE, float>(a, b, cm, M, N, K, ep, err, num_sms, st);
+      return launch_tc2<224, EPI_STORE, float>(a, b, cm, pm, M, N, K, ep, err, num_sms, st);
     return cudaErrorInvalidValue;
   }
   if (out_bf16) {

@@ -37,14 +37,16 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // bf16 tensor-core GEMM (gemm_tc.cu): out = epilogue(A[M,K] * W[N,K]^T); `a`, `b`
 // are TMA maps of A (box 64 x 128) and W (box 64 x bn, or 64 x bn/2 when `pair`) with
 // the 128-byte swizzle. N % bn == 0, K % 64 == 0. `pair`: 256 x bn tiles computed by
-// two CTAs of a cluster with cta_group::2 (bn == 256, N <= 4096 and 4 x tiles <= num_sms:
-// one tile per cluster of four, K split over two such pairs); their epilogues store through `c`, a TMA map of
-// the output (EPI_RESID: of the fp32 residual; EPI_QKV: 3D [3*B*heads][L][128]) with box
-// 32 x 32 (x 1) and the 128-byte (fp32) or 64-byte (bf16) swizzle.
+// two CTAs of a cluster with cta_group::2, persistent over every CTA pair; their epilogues
+// store through `c`, a TMA map of the output (EPI_RESID: of the fp32 residual; EPI_QKV: 3D
+// [3*B*heads][L][128]) with box 32 x 32 (x 1) and the 128-byte (fp32) or 64-byte (bf16)
+// swizzle. With ep.sk_part set the pairs split the k-blocks stream-K: `p` is then a 2D fp32
+// map of the partial-sum slots [pairs * 256 rows][256] with box 32 x 32 and the 128-byte
+// swizzle, and ep.sk_flags the per-(tile, CTA, quarter) counters, zero on entry.
 cudaError_t gemm_tc_prepare();  // sets the kernels' shared-memory attributes on the current device
-cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, int M, int N, int K, int bn,
-                    int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
-                    bool pair = false);
+cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, const CUtensorMap* p, int M,
+                    int N, int K, int bn, int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms,
+                    cudaStream_t st, bool pair = false);
 
 // fp32 CUDA-core GEMM (misc.cu) with the same epilogues; N % 128 == 0.
 cudaError_t gemm_simt(const float* A, long lda, const float* W, long ldw, int M, int N, int K, int kind,
@@ -121,5 +123,14 @@ cudaError_t gen_tensor(T* dst, long rows, long cols, long ld, uint64_t seed, int
 cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st);
 cudaError_t fill_f32(float* p, long n, float v, cudaStream_t st);
 cudaError_t wait_probe(unsigned* err, cudaStream_t st);
+
+// audio projection (audio.cu): gather the encoder states each latent frame reads, and a
+// skinny split-K product y = act(x W^T + b) with an output row map (see audio.cu)
+cudaError_t audio_windows(const float* states, float* win0, float* winv, int batch, int S, int per_state, int F,
+                          int s0, int window, int stride, int group, cudaStream_t st);
+int audio_gemv_chunks(int K);
+template <typename WT>
+cudaError_t audio_linear(const WT* W, const float* x, const float* bias, float* part, float* y, int N, int K, int R,
+                         int relu, int per, int ostride, int ooff, cudaStream_t st);
 
 }  // namespace fh

@@ -6,17 +6,15 @@
 
 #include "epilogue.cuh"
 #include "kernels.h"
+#include "rownorm.cuh"
 
 namespace fh {
 
 namespace {
 
 // ------------------------------------------------------------------ row norms
-// One warp per row; D = 128 * NV floats held in registers (float4 per lane per step).
-// Mode 0 / 2: the adaLN modulate h = n(x) * (1 + scale) + shift of the Wan-style
-// block (reading R1) and of the output norm (headMods, gizai:flashhead Types >
-// FlashHead, reading R9); mode 1: the learned-affine LayerNorm before the audio
-// cross-attention (reading R7). Biased variance, eps inside the root (R2).
+// One warp per row (rownorm.cuh): the adaLN modulate of the block and of the output norm
+// (modes 0, 2) and the learned-affine LayerNorm before the audio cross-attention (mode 1).
 template <typename T, int NV>
 __global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ out, int M, int rows_per_batch,
                                  int mode, const float* __restrict__ shift, const float* __restrict__ scale,
@@ -28,64 +26,9 @@ __global__ void norm_rows_kernel(const float* __restrict__ x, T* __restrict__ ou
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
-  const float4* xr = reinterpret_cast<const float4*>(x + (long)row * D);
-  float4 v[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) v[i] = xr[lane + 32 * i];
-  // the affine / modulation vectors are loaded alongside the row, before the reductions
   const long mb = (long)(row / rows_per_batch) * mod_bstride;
-  const float* av = mode == 1 ? w : scale + mb;
-  const float* cv = mode == 1 ? bb : shift + mb;
-  float4 ma[NV], mc[NV];
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    ma[i] = reinterpret_cast<const float4*>(av)[lane + 32 * i];
-    mc[i] = reinterpret_cast<const float4*>(cv)[lane + 32 * i];
-  }
-  float mu = 0.f, rstd;
-  if (mode != 2) {
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-    mu = warp_sum(s) * (1.f / D);
-    float q = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const float a = v[i].x - mu, b = v[i].y - mu, c = v[i].z - mu, d = v[i].w - mu;
-      q += (a * a + b * b) + (c * c + d * d);
-    }
-    rstd = rsqrtf(warp_sum(q) * (1.f / D) + eps);
-  } else {
-    float q = 0.f;
-#pragma unroll
-    for (int i = 0; i < NV; ++i) q += (v[i].x * v[i].x + v[i].y * v[i].y) + (v[i].z * v[i].z + v[i].w * v[i].w);
-    rstd = rsqrtf(warp_sum(q) * (1.f / D) + eps);
-  }
-  T* orow = out + (long)row * D;
-#pragma unroll
-  for (int i = 0; i < NV; ++i) {
-    const int col = (lane + 32 * i) * 4;
-    float y[4] = {(v[i].x - mu) * rstd, (v[i].y - mu) * rstd, (v[i].z - mu) * rstd, (v[i].w - mu) * rstd};
-    float4 a = ma[i];
-    const float4 c = mc[i];
-    if (mode != 1) {
-      a.x += 1.f; a.y += 1.f; a.z += 1.f; a.w += 1.f;
-    }
-    y[0] = y[0] * a.x + c.x;
-    y[1] = y[1] * a.y + c.y;
-    y[2] = y[2] * a.z + c.z;
-    y[3] = y[3] * a.w + c.w;
-    if constexpr (sizeof(T) == 2) {
-      __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
-      __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
-      uint2 u;
-      u.x = *reinterpret_cast<uint32_t*>(&h0);
-      u.y = *reinterpret_cast<uint32_t*>(&h1);
-      *reinterpret_cast<uint2*>(orow + col) = u;
-    } else {
-      *reinterpret_cast<float4*>(orow + col) = make_float4(y[0], y[1], y[2], y[3]);
-    }
-  }
+  norm_row<T, NV>(x + (long)row * D, out + (long)row * D, lane, mode, mode == 1 ? w : scale + mb,
+                  mode == 1 ? bb : shift + mb, eps);
 }
 
 // ------------------------------------------------------ per-frame cross-attention
@@ -454,22 +397,22 @@ __global__ void gen_tensor_kernel(T* __restrict__ dst, long rows, long cols, lon
 // [pf, pf+ph) with the row, the rest with the column; pair j of an axis with n dims
 // turns theta^(-2j/n) rad per position (reading R3; table shape as the `cos`/`sin`
 // fields of gizai:flashhead Types > FlashHead, one head's 64 columns).
+// Rotary (cos, sin) per axis (reading R3): [F][pf] by frame index, [H][ph] by row, [W][pw] by
+// column, one after the other; pair j of an axis of n = 2 * (pairs) dims at position pos turns
+// pos * theta^(-2j / n) radians (float64, then rounded to float32).
 __global__ void rope_table_kernel(float2* tab, int F, int H, int W, int pf, int ph, int pw, double theta) {
   pdl_launch_dependents();
   pdl_wait();
-  const int L = F * H * W;
-  const int np = pf + ph + pw;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= L * np) return;
-  const int n = idx / np, d = idx % np;
-  const int f = n / (H * W), r = (n / W) % H, c = n % W;
+  const int nf = F * pf, nh = H * ph, nw = W * pw;
+  if (idx >= nf + nh + nw) return;
   int pos, j, ndim;
-  if (d < pf) {
-    pos = f; j = d; ndim = 2 * pf;
-  } else if (d < pf + ph) {
-    pos = r; j = d - pf; ndim = 2 * ph;
+  if (idx < nf) {
+    pos = idx / pf; j = idx % pf; ndim = 2 * pf;
+  } else if (idx < nf + nh) {
+    pos = (idx - nf) / ph; j = (idx - nf) % ph; ndim = 2 * ph;
   } else {
-    pos = c; j = d - pf - ph; ndim = 2 * pw;
+    pos = (idx - nf - nh) / pw; j = (idx - nf - nh) % pw; ndim = 2 * pw;
   }
   const double ang = (double)pos * pow(theta, -2.0 * (double)j / (double)ndim);
   tab[idx] = make_float2((float)cos(ang), (float)sin(ang));
@@ -693,7 +636,7 @@ template cudaError_t gen_tensor<float>(float*, long, long, long, uint64_t, int, 
 template cudaError_t gen_tensor<bf16>(bf16*, long, long, long, uint64_t, int, int, int, bool, cudaStream_t);
 
 cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st) {
-  const int n = F * H * W * (pf + ph + pw);
+  const int n = F * pf + H * ph + W * pw;
   { cudaError_t e_ = launch_pdl(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, st, tab, F, H, W, pf, ph, pw, (double)theta); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }

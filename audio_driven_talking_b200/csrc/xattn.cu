@@ -89,6 +89,9 @@ __global__ void __launch_bounds__(XT_THREADS, 1)
     tmem_alloc(tmem_holder, XT_TMEM_COLS);
     tmem_relinquish();
   }
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -232,6 +235,9 @@ __global__ void __launch_bounds__(XT_THREADS, 1)
     }
   }
 
+  // every role ends here with its warp converged again (a lane that did a role's work arrives
+  // after the others), so the CTA barrier below counts each warp once, after all of its work
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -100,9 +100,14 @@ typedef struct fh_dit fh_dit;
  * even) for FH_BF16 models. */
 #define FH_BLOCK_TENSOR(k, s) (64 * (k) + (s))
 #define FH_GLOBAL_TENSOR(g) (4096 + (g))
+/* Audio projection tensors (fh_audio_project), id 4096 + 32 + a, HID = 512, K0 = 5 * 12 * 768,
+ * KV = 12 * 12 * 768: 0 proj1_w[HID,K0] 1 proj1_b[HID] 2 proj1vf_w[HID,KV] 3 proj1vf_b[HID]
+ * 4 proj2_w[HID,HID] 5 proj2_b[HID] 6 proj3_w[32D,HID] 7 proj3_b[32D] 8 projnorm_w[D] (a gain)
+ * 9 projnorm_b[D] (a LayerNorm bias). */
+#define FH_AUDIO_TENSOR(a) (4096 + 32 + (a))
 
 /* Create a model on cfg->device: allocates and owns the weights (generated on the
- * GPU from `seed`), the rotary table [L, 64] and internal buffers. Synchronises
+ * GPU from `seed`), the rotary tables (cos, sin per axis) and internal buffers. Synchronises
  * `stream` before returning. Errors: FH_ERR_ARG (null), FH_ERR_SHAPE (config
  * constraints), FH_ERR_UNSUPPORTED (not sm_100), FH_ERR_OOM, FH_ERR_CUDA. */
 int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** out);
@@ -165,6 +170,21 @@ int fh_sample_slice_host(fh_dit* m, const float* noise_host, const float* ref_ho
                          const float* motion_host, const void* audio_host,
                          const float* sigmas, int nsteps, float* x_out_host, int batch,
                          void* ws, void* stream);
+
+/* The audio projection of one slice (gizai:flashhead, opening paragraph: the last 8 s of
+ * speech through wav2vec 2.0 base, its 12 layers' states at 200 frames; 5 states around each
+ * of the slice's 33 frames make 5 latent frames of 32 audio tokens; Types > FlashHead: proj1,
+ * proj1vf, proj2, proj3, projNorm). states: device float32 [B, 200, 12, 768], the encoder's
+ * states over the audio window (the last of them at the slice's last video frame). tokens:
+ * device [B, frames, 32, dim] in the model dtype, the `audio` argument of the calls above.
+ * Video frame t of the slice's 1 + 8 (frames - 1) takes the states within two of state
+ * 200 - (1 + 8 (frames - 1)) + t (clamped to the window); latent frame 0 reads video frame
+ * 0's 5 states through proj1, latent frame j >= 1 the 12 states spanning video frames
+ * 8j-7..8j through proj1vf; both with a ReLU, then proj2 with a ReLU, proj3 to 32 tokens and
+ * projNorm, a LayerNorm with weight and bias over each token. Asynchronous on `stream`; uses
+ * the workspace. Errors: as fh_dit_block_forward; FH_ERR_SHAPE if the latent frames need more
+ * than 200 states. */
+int fh_audio_project(fh_dit* m, const float* states, void* tokens, int batch, void* ws, void* stream);
 
 /* Copy weight tensor `tensor_id` to host memory as float32 in its logical
  * row-major shape; `bytes` must equal 4 * element count. Synchronous. */

@@ -23,14 +23,56 @@ extern "C" {
 int fh_op_linear(const void* A, const void* W, const float* bias, float* out, int M, int N, int K, int dtype,
                  void* stream);
 
+/* fh_op_linear (dtype FH_BF16) on 256-row CTA-pair tiles with the k-blocks of all tiles
+ * split evenly over every CTA pair of the GPU (stream-K), the way the model's block
+ * projections run: a tile cut between pairs is finished by the pair holding its first
+ * k-blocks, which adds the others' fp32 partial sums in k order (deterministic). Only for
+ * shapes that run on CTA pairs (K >= 1024, 1536 <= N <= 16384, N % 128 == 0, K % 64 == 0;
+ * else FH_ERR_SHAPE). ws: caller-owned device scratch, 256-byte aligned, of at least
+ * fh_op_linear_streamk_bytes(M, N, K) bytes (else FH_ERR_ARG; the call clears the part that
+ * must start at zero); calls sharing a ws must not overlap in time.
+ * fh_op_linear_streamk_bytes returns 0 for an invalid shape. */
+size_t fh_op_linear_streamk_bytes(int M, int N, int K);
+int fh_op_linear_streamk(const void* A, const void* W, const float* bias, float* out, int M, int N, int K, void* ws,
+                         size_t ws_bytes, void* stream);
+
 /* Non-causal self-attention over L tokens per (stream, head), as inside a block
  * (gizai:flashhead, opening paragraph; readings R4-R6): q, k, v [batch, heads, L,
- * 128] in dtype; ssq float32 [batch*L, 2*heads] with the per-head partial sums of
+ * 128] in dtype, except that with FH_BF16 v is float16 (as the QKV projection stores it:
+ * the kernel multiplies v by float16 softmax weights); ssq float32 [batch*L, 2*heads] with the per-head partial sums of
  * squares of q (first heads columns) and k (last heads columns), whose sum over
  * heads divided by heads*128, plus eps, gives each token's RMS factor r^-2; scores
  * are r_i r_j (q_i . k_j) / sqrt(128). out [batch*L, heads*128] in dtype. */
 int fh_op_attention(const void* q, const void* k, const void* v, const float* ssq, void* out, int batch,
                     int heads, int L, float eps, int dtype, void* stream);
+
+/* Per-frame audio cross-attention, as inside a block (gizai:flashhead, opening paragraph:
+ * each slice's audio becomes 5 latent frames of 32 audio tokens; readings R4-R6): token n
+ * of latent frame f = n / hw of stream b attends to the audio_tokens (= 32, else
+ * FH_ERR_SHAPE) keys of that frame only,
+ *   out_n = sum_a softmax_a(r_n r_a (q_n . k_a) / sqrt(128)) v_a   per head.
+ * q [batch*frames*hw, heads*128] (token-major, frame-major within a stream) in dtype;
+ * ssq_q float32 [batch*frames*hw, heads] per-head partial sums of squares of the query
+ * row, whose sum over heads divided by heads*128, plus eps, gives r_n^-2; kv
+ * [batch*frames*32, 2*heads*128] in dtype: row (b*frames + f)*32 + a holds key a of that
+ * frame in its first heads*128 columns and its value in the rest; ssq_k float32
+ * [batch*frames*32, heads] the keys' partial sums. out like q. dtype FH_BF16: the
+ * tensor-core kernel (TMA over 3D [frame][hw][D] views: hw need not be a multiple of
+ * 128, rows past a frame are neither read nor written); FH_F32: CUDA cores. */
+int fh_op_cross_attention(const void* q, const float* ssq_q, const void* kv, const float* ssq_k, void* out,
+                          int batch, int heads, int frames, int hw, int audio_tokens, float eps, int dtype,
+                          void* stream);
+
+/* One norm and modulation per row, as before the block's projections (gizai:flashhead,
+ * opening paragraph, "Wan-style"; readings R1, R2, R7, R9): x float32 [M, D] (D / 128 in
+ * {1, 2, 3, 4, 6, 8, 12, 16}, else FH_ERR_SHAPE), out [M, D] in dtype.
+ *   mode 0: LayerNorm(x) * (1 + a) + c    mode 2: RMSNorm(x) * (1 + a) + c
+ *     (a = scale, c = shift: float32 vectors of D, the stream's own at a + (row /
+ *      rows_per_batch) * bstride)
+ *   mode 1: LayerNorm(x) * a + c            (a = weight, c = bias; bstride ignored)
+ * LayerNorm with the biased variance, no gain of its own; eps inside the root. */
+int fh_op_row_norm(const float* x, void* out, int M, int D, int mode, const float* a, const float* c, long bstride,
+                   int rows_per_batch, float eps, int dtype, void* stream);
 
 /* Failure-detection check (no counterpart on the pages; reading of the pages'
  * reject-don't-hang stance): launches one CTA whose mbarrier wait has no arriving
