@@ -537,15 +537,6 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec*
     ep.norm_period = 3 * D;
     ep.norm_count = 2 * D;
     ep.rope = m->rope;
-    {
-      const int pf = m->cfg.rope_split[0] / 2, ph = m->cfg.rope_split[1] / 2;
-      ep.rope_H = m->cfg.lat_h;
-      ep.rope_W = m->cfg.lat_w;
-      ep.rope_pf = pf;
-      ep.rope_ph = ph;
-      ep.rope_off_h = m->F * pf;
-      ep.rope_off_w = m->F * pf + m->cfg.lat_h * ph;
-    }
     ep.dim = D;
     ep.sec_stride = (long)M * D;
     RUN(run_gemm(m, &P.m_h, h, D, &bw.m_qkv, bw.wqkv, D, M, 3 * D, D, EPI_QKV, m->bf16, ep, st, 3));
@@ -808,7 +799,7 @@ int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** ou
                o_mod = take(NB * 6 * D * 4), o_pw = take(D * 2 * C * e), o_pb = take(D * 4), o_hw = take(C * D * e),
                o_hb = take(C * 4), o_hm = take(2 * D * 4), o_tw1 = take(D * 256 * e), o_tb1 = take(D * 4),
                o_tw2 = take(D * D * e), o_tb2 = take(D * 4), o_twp = take(6 * D * D * e), o_tbp = take(6 * D * 4),
-               o_rope = take((size_t)(c.frames + c.lat_h + c.lat_w) * 64 * 8);
+               o_rope = take((size_t)L * 64 * 8);
   const size_t o_aw1 = take((size_t)AU_HID * AU_K0 * e), o_ab1 = take(AU_HID * 4),
                o_aw1v = take((size_t)AU_HID * AU_KV * e), o_ab1v = take(AU_HID * 4),
                o_aw2 = take((size_t)AU_HID * AU_HID * e), o_ab2 = take(AU_HID * 4),

@@ -42,10 +42,7 @@ struct EpiParams {
   int ssq_ld;
   int norm_period;        // column c is normed iff (c % norm_period) < norm_count
   int norm_count;
-  // EPI_QKV: the rotary (cos, sin) per axis: [F][pf] for the frame index, then [H][ph] for the
-  // row, then [W][pw] for the column (pf + ph + pw = 64 pairs); token l = (f H + r) W + c
-  const float2* rope;
-  int rope_H, rope_W, rope_pf, rope_ph, rope_off_h, rope_off_w;
+  const float2* rope;     // EPI_QKV: (cos, sin) [rows_per_batch, 64]
   int dim;                // EPI_QKV: width D of each of the q, k, v sections
   long sec_stride;        // EPI_QKV: elements per section = B * heads * L * 128
   // CTA-pair GEMM, stream-K: fp32 partial sums [clusters][2][128][BN] and per-(tile, CTA,
@@ -117,27 +114,40 @@ __device__ __forceinline__ void epi_math(const EpiParams& p, int row, int col0, 
 }
 
 // EPI_QKV on q and k columns: rotate adjacent pairs (2d, 2d+1) by the angles of the row's
-// token position. A pair turns with one axis only (reading R3), so its (cos, sin) comes from
-// that axis's small table (a few KB: it stays in L1 for every row of a tile).
+// token position (table (cos, sin) [rows_per_batch, 64]).
 __device__ __forceinline__ void epi_rope(const EpiParams& p, int row, int col0, float (&v)[32]) {
   const int l = row % p.rows_per_batch;
-  const int hw = p.rope_H * p.rope_W;
-  const int f = l / hw, r = (l / p.rope_W) % p.rope_H, c = l % p.rope_W;
-  const int pf = p.rope_pf, pfh = p.rope_pf + p.rope_ph, pw = 64 - pfh;
-  const int pair0 = ((col0 % p.dim) & 127) >> 1;
+  const int d0 = (col0 % p.dim) & 127;
+  const float2* rt = p.rope + (long)l * 64 + (d0 >> 1);
 #pragma unroll
   for (int j = 0; j < 32; j += 2) {
-    const int d = pair0 + (j >> 1);  // the same for every lane
-    float2 cs;
-    if (d < pf)
-      cs = p.rope[f * pf + d];
-    else if (d < pfh)
-      cs = p.rope[p.rope_off_h + r * p.rope_ph + (d - pf)];
-    else
-      cs = p.rope[p.rope_off_w + c * pw + (d - pfh)];
+    float2 cs = rt[j >> 1];
     float x0 = v[j], x1 = v[j + 1];
     v[j] = x0 * cs.x - x1 * cs.y;
     v[j + 1] = x0 * cs.y + x1 * cs.x;
+  }
+}
+
+// EPI_QKV: the (cos, sin) of the 16 rotary pairs of columns [col0, col0 + 32) of `row`, loaded
+// ahead of their use (the table rows of a tile's 128 rows do not fit in L1, so these are L2
+// reads whose latency the previous chunk's work hides).
+__device__ __forceinline__ void epi_rope_load(const EpiParams& p, int row, int col0, float4 (&cs)[8]) {
+  const int l = row % p.rows_per_batch;
+  const float4* rt = reinterpret_cast<const float4*>(p.rope + (long)l * 64 + (((col0 % p.dim) & 127) >> 1));
+#pragma unroll
+  for (int k = 0; k < 8; ++k) cs[k] = rt[k];
+}
+// epi_rope with the pairs' (cos, sin) already in registers
+__device__ __forceinline__ void epi_rope_apply(const float4 (&cs)[8], float (&v)[32]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float x0 = v[4 * k], x1 = v[4 * k + 1];
+    v[4 * k] = x0 * cs[k].x - x1 * cs[k].y;
+    v[4 * k + 1] = x0 * cs[k].y + x1 * cs[k].x;
+    x0 = v[4 * k + 2];
+    x1 = v[4 * k + 3];
+    v[4 * k + 2] = x0 * cs[k].z - x1 * cs[k].w;
+    v[4 * k + 3] = x0 * cs[k].w + x1 * cs[k].z;
   }
 }
 
@@ -158,9 +168,9 @@ __device__ __forceinline__ void epi_prefetch(const EpiParams& p, int row, int co
       if (epi_normed(p, col0 + c)) prefetch_l1(p.gain + col0 + c);
     }
   }
-  if constexpr (KIND == EPI_QKV) {  // the rotary tables (a few KB): one 128-byte line per lane
-    const int n = p.rope_off_w + p.rope_W * (64 - p.rope_pf - p.rope_ph);
-    for (int i = (threadIdx.x & 31) * 16; i < n; i += 32 * 16) prefetch_l1(p.rope + i);
+  if constexpr (KIND == EPI_QKV) {  // the row's rotary angles (64 (cos, sin) pairs, 4 lines)
+    const float2* rt = p.rope + (long)(row % p.rows_per_batch) * 64;
+    for (int c = 0; c < 64; c += 16) prefetch_l1(rt + c);
   }
 }
 

@@ -586,6 +586,20 @@ __global__ void __launch_bounds__(192, 1)
       // whole tile, or the owner of a cut tile: wait for its contributors' partial sums
       const int ncontrib = (R.sk && sg.kb1 < nk) ? R.contributors(sg.tile, cl) : 0;
       epi_prefetch<KIND>(ep, row < M ? row : M - 1, n0, BN);  // while the MMAs run
+      // EPI_QKV: the 32 rows stay inside one stream (row0 and L both multiples of 32 at
+      // the usual sizes); otherwise this warp stores directly, row by row
+      bool direct = false;
+      int l0 = 0, bidx = 0;
+      if constexpr (KIND == EPI_QKV) {
+        l0 = row0 % ep.rows_per_batch;
+        bidx = row0 / ep.rows_per_batch;
+        direct = l0 + 32 > ep.rows_per_batch && row0 + (ep.rows_per_batch - l0) < M;
+      }
+      // EPI_QKV: the rotary (cos, sin) of the next chunk, loaded one chunk ahead (the first
+      // chunk's while the MMAs run)
+      float4 rope_cur[8], rope_nxt[8];
+      const bool rope_rows = KIND == EPI_QKV && row0 < M && !direct;
+      if (rope_rows && epi_normed(ep, n0)) epi_rope_load(ep, row < M ? row : M - 1, n0, rope_cur);
       bool ok = mbar_wait(&tfull[acc], aph, abort_flag, err, ERRBIT_TIMEOUT_GEMM);
       if (ncontrib > 0 && lane == 0 && ok) {
         const uint64_t t0 = globaltimer();
@@ -622,18 +636,11 @@ __global__ void __launch_bounds__(192, 1)
         for (; nissued < nbox && nissued < S::PBOX; ++nissued) issue_box(nissued);
       int nwait = 0;
       bool pok = true;  // every box arrived in time
-      // EPI_QKV: the 32 rows stay inside one stream (row0 and L both multiples of 32 at
-      // the usual sizes); otherwise this warp stores directly, row by row
-      bool direct = false;
-      int l0 = 0, bidx = 0;
-      if constexpr (KIND == EPI_QKV) {
-        l0 = row0 % ep.rows_per_batch;
-        bidx = row0 / ep.rows_per_batch;
-        direct = l0 + 32 > ep.rows_per_batch && row0 + (ep.rows_per_batch - l0) < M;
-      }
       // one 32-column chunk of the tile: contributors' partial sums, the epilogue, the store
       float ssq = 0.f;
       auto chunk = [&](float (&v)[32], int c) {
+        if (rope_rows && c + 32 < BN && epi_normed(ep, n0 + c + 32))
+          epi_rope_load(ep, row < M ? row : M - 1, n0 + c + 32, rope_nxt);
         // contributors' partial sums of these 32 columns, in k order
         for (int q = 0; q < ncontrib && pok; ++q, ++nwait) {
           const int slot = nwait % S::PBOX;
@@ -659,7 +666,7 @@ __global__ void __launch_bounds__(192, 1)
           if (row < M) {
             epi_math<KIND, OutT>(ep, row, n0 + c, v, ssq);
             if constexpr (KIND == EPI_QKV)
-              if (epi_normed(ep, n0 + c)) epi_rope(ep, row, n0 + c, v);
+              if (epi_normed(ep, n0 + c)) epi_rope_apply(rope_cur, v);
           } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -695,20 +702,17 @@ __global__ void __launch_bounds__(192, 1)
           if (row < M) epi_group_end<KIND>(ep, row, n0 + (c & ~127), ssq);
           ssq = 0.f;
         }
+        if constexpr (KIND == EPI_QKV) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) rope_cur[k] = rope_nxt[k];
+        }
       };
-      // the accumulator's chunks leave TMEM one ahead of their use: each wait covers the
-      // chunk loaded while the previous one was being processed
-      float va[32], vb[32];
-      tmem_ld32(tb, va);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 64) {
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld32(tb + c, v);
         tc_wait_ld();
-        if (c + 32 < BN) tmem_ld32(tb + c + 32, vb);
-        chunk(va, c);
-        if (c + 32 >= BN) break;
-        tc_wait_ld();
-        if (c + 64 < BN) tmem_ld32(tb + c + 64, va);
-        chunk(vb, c + 32);
+        chunk(v, c);
       }
       if (!pok) {
         // boxes still in flight land before the CTA's shared memory can go away
@@ -991,17 +995,12 @@ __global__ void __launch_bounds__(192, 1)
           *reinterpret_cast<float4*>(prow + ((j ^ (lane & 7)) << 4)) =
               make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
       };
-      // chunks leave TMEM one ahead of their use (HALF_COLS is a multiple of 64)
-      float va[32], vb[32];
-      tmem_ld32(tb + theirs, va);
 #pragma unroll 1
-      for (int c = 0; c < (int)HALF_COLS; c += 64) {
+      for (int c = 0; c < (int)HALF_COLS; c += 32) {
+        float v[32];
+        tmem_ld32(tb + theirs + c, v);
         tc_wait_ld();
-        tmem_ld32(tb + theirs + c + 32, vb);
-        put(va, c);
-        tc_wait_ld();
-        if (c + 64 < (int)HALF_COLS) tmem_ld32(tb + theirs + c + 64, va);
-        put(vb, c + 32);
+        put(v, c);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -1050,17 +1049,12 @@ __global__ void __launch_bounds__(192, 1)
         }
         ++nchunk;
       };
-      // chunks leave TMEM one ahead of their use
-      float va[32], vb[32];
-      tmem_ld32(tb + mine, va);
 #pragma unroll 1
-      for (int c = 0; c < (int)HALF_COLS; c += 64) {
+      for (int c = 0; c < (int)HALF_COLS; c += 32) {
+        float v[32];
+        tmem_ld32(tb + mine + c, v);
         tc_wait_ld();
-        tmem_ld32(tb + mine + c + 32, vb);
-        chunk(va, c);
-        tc_wait_ld();
-        if (c + 64 < (int)HALF_COLS) tmem_ld32(tb + mine + c + 64, va);
-        chunk(vb, c + 32);
+        chunk(v, c);
       }
       if (row < M) epi_group_end<KIND>(ep, row, n0 + mine, ssq);
     }

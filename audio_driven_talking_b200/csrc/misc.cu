@@ -403,16 +403,19 @@ __global__ void gen_tensor_kernel(T* __restrict__ dst, long rows, long cols, lon
 __global__ void rope_table_kernel(float2* tab, int F, int H, int W, int pf, int ph, int pw, double theta) {
   pdl_launch_dependents();
   pdl_wait();
+  const int L = F * H * W;
+  const int np = pf + ph + pw;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  const int nf = F * pf, nh = H * ph, nw = W * pw;
-  if (idx >= nf + nh + nw) return;
+  if (idx >= L * np) return;
+  const int n = idx / np, d = idx % np;
+  const int f = n / (H * W), r = (n / W) % H, c = n % W;
   int pos, j, ndim;
-  if (idx < nf) {
-    pos = idx / pf; j = idx % pf; ndim = 2 * pf;
-  } else if (idx < nf + nh) {
-    pos = (idx - nf) / ph; j = (idx - nf) % ph; ndim = 2 * ph;
+  if (d < pf) {
+    pos = f; j = d; ndim = 2 * pf;
+  } else if (d < pf + ph) {
+    pos = r; j = d - pf; ndim = 2 * ph;
   } else {
-    pos = (idx - nf - nh) / pw; j = (idx - nf - nh) % pw; ndim = 2 * pw;
+    pos = c; j = d - pf - ph; ndim = 2 * pw;
   }
   const double ang = (double)pos * pow(theta, -2.0 * (double)j / (double)ndim);
   tab[idx] = make_float2((float)cos(ang), (float)sin(ang));
@@ -636,7 +639,7 @@ template cudaError_t gen_tensor<float>(float*, long, long, long, uint64_t, int, 
 template cudaError_t gen_tensor<bf16>(bf16*, long, long, long, uint64_t, int, int, int, bool, cudaStream_t);
 
 cudaError_t rope_table(float2* tab, int F, int H, int W, int pf, int ph, int pw, float theta, cudaStream_t st) {
-  const int n = F * pf + H * ph + W * pw;
+  const int n = F * H * W * (pf + ph + pw);
   { cudaError_t e_ = launch_pdl(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, st, tab, F, H, W, pf, ph, pw, (double)theta); if (e_ != cudaSuccess) return e_; }
   return cudaGetLastError();
 }

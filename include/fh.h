@@ -107,7 +107,7 @@ typedef struct fh_dit fh_dit;
 #define FH_AUDIO_TENSOR(a) (4096 + 32 + (a))
 
 /* Create a model on cfg->device: allocates and owns the weights (generated on the
- * GPU from `seed`), the rotary tables (cos, sin per axis) and internal buffers. Synchronises
+ * GPU from `seed`), the rotary table [L, 64] and internal buffers. Synchronises
  * `stream` before returning. Errors: FH_ERR_ARG (null), FH_ERR_SHAPE (config
  * constraints), FH_ERR_UNSUPPORTED (not sm_100), FH_ERR_OOM, FH_ERR_CUDA. */
 int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** out);
