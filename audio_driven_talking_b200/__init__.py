@@ -112,8 +112,6 @@ def load_library() -> ctypes.CDLL:
         "fh_op_attention": (I, [P, P, P, P, P, I, I, I, F, I, P]),
         "fh_op_cross_attention": (I, [P, P, P, P, P, I, I, I, I, I, F, I, P]),
         "fh_op_row_norm": (I, [P, P, I, I, I, P, P, ctypes.c_long, I, F, I, P]),
-        "fh_op_linear_streamk_bytes": (Z, [I, I, I]),
-        "fh_op_linear_streamk": (I, [P, P, P, P, I, I, I, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -290,21 +288,6 @@ def linear(A, W, bias, stream=None):
     return out
 
 
-def linear_streamk(A, W, bias, stream=None):
-    """linear() for bf16 CTA-pair shapes with the stream-K split of the model's block GEMMs."""
-    import torch
-    M, K = A.shape
-    N = W.shape[0]
-    lib = load_library()
-    n = int(lib.fh_op_linear_streamk_bytes(M, N, K))
-    if n == 0:
-        raise FHError(FH_ERR_SHAPE, f"bad GEMM shape {M} x {N} x {K}")
-    ws = torch.empty(n, dtype=torch.uint8, device=A.device)
-    out = torch.empty((M, N), dtype=torch.float32, device=A.device)
-    _check(lib.fh_op_linear_streamk(_ptr(A), _ptr(W), _ptr(bias), _ptr(out), M, N, K, _ptr(ws), n, _stream(stream)))
-    return out
-
-
 def cross_attention(q, ssq_q, kv, ssq_k, frames, eps=1e-6, stream=None):
     """Per-frame audio cross-attention (see include/fh_ops.h): q [B, frames*hw, heads*128],
     kv [B, frames, 32, 2*heads*128] (keys then values), ssq_q/ssq_k float32 per-head sums."""
@@ -342,4 +325,4 @@ def attention(q, k, v, ssq, eps=1e-6, stream=None):
 
 
 __all__ = ["DiT", "ModelConfig", "LITE", "FP32_BLOCK", "ONE_BLOCK", "LITE_768_X3", "FHError", "load_library",
-           "linear", "linear_streamk", "attention", "cross_attention", "row_norm", "FH_F32", "FH_BF16"]
+           "linear", "attention", "cross_attention", "row_norm", "FH_F32", "FH_BF16"]

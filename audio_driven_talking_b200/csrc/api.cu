@@ -124,14 +124,12 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Tile shape per GEMM, from the weight's N and K. Deep projections (K >= 1024, N >= 1536:
 // QKV, O-proj, cross-Q/O, FFN1, FFN2) run as 256-row tiles on CTA pairs (cta_group::2),
 // each CTA streaming half of the W tile, 256 columns wide where N allows (the widest tile
-// a pair accumulates, the least operand traffic per MMA), with a stream-K split of the
-// k-blocks over all CTA pairs so that no round of tiles runs part-empty; the rest (patch
-// embed K = 256, head N = 128, the per-slice cross-KV with 160 rows) on single CTAs.
+// a pair accumulates, the least operand traffic per MMA); the rest (patch embed K = 256,
+// head N = 128, the per-slice cross-KV with 160 rows) on single CTAs.
 struct TileCfg {
   int bn;
   bool pair;
-  bool streamk;  // split the k-blocks over every CTA pair (else whole tiles per pair)
-  int wbox;      // rows of the W tile each CTA loads
+  int wbox;  // rows of the W tile each CTA loads
 };
 TileCfg tile_cfg(int N, int K, bool pair_ok = true) {
   TileCfg t;
@@ -143,7 +141,6 @@ TileCfg tile_cfg(int N, int K, bool pair_ok = true) {
   // FFN1 (N = 8960 = 40 x 224): at 1280 tokens 200 pair tiles of width 224 fill three rounds
   // of 74 CTA pairs better than 175 tiles of width 256
   if (t.pair && N >= 8192 && N % 224 == 0) t.bn = 224;
-  t.streamk = false;
   t.wbox = t.pair ? t.bn / 2 : t.bn;
   return t;
 }
@@ -155,9 +152,6 @@ constexpr int AU_STATES = 200, AU_LAYERS = 12, AU_CH = 768, AU_WIN = 5, AU_STRID
 constexpr int AU_PER_STATE = AU_LAYERS * AU_CH;
 constexpr int AU_GROUP = AU_STRIDE + AU_WIN - 1;
 constexpr int AU_K0 = AU_WIN * AU_PER_STATE, AU_KV = AU_GROUP * AU_PER_STATE;
-
-constexpr bool kFuseNorms = false;  // norm of the finished rows inside the gated-residual GEMM
-constexpr int LN_COUNTERS = 8192;  // fused-norm launches per call (a 64-step slice of 30 blocks needs 5760)
 
 struct TensorRec {
   int tid;
@@ -176,7 +170,7 @@ struct BlockW {
 
 struct WsLayout {
   size_t x, h, qkv, ssq_qk, attn, cq, ssq_cq, ckv, ssq_ckv, u, tok, lat, v, mods, hmods, tsin, thid, te, te0, audio,
-      in_noise, in_ref, in_motion, out, sk_part, sk_flags, sk_flags_bytes, ln_ctr, au_win0, au_winv, au_part, au_h1, au_h2,
+      in_noise, in_ref, in_motion, out, au_win0, au_winv, au_part, au_h1, au_h2,
       au_tok, total;
 };
 
@@ -186,7 +180,6 @@ struct Plan {
   WsLayout lay{};
   CUtensorMap m_h, m_attn, m_u, m_tok, m_audio, m_q, m_k, m_v;
   CUtensorMap m_xq, m_xkv, m_xo;  // cross-attention: queries and output per frame, keys/values
-  CUtensorMap m_skp;              // stream-K partial-sum slots of the CTA-pair GEMMs
 };
 
 struct GraphEntry {
@@ -227,7 +220,6 @@ struct fh_dit {
   std::vector<GraphEntry> graphs;
   cudaStream_t cap = nullptr;
   int launches = 0, last_launches = 0;
-  int ln_seq = 0;  // fused-norm counters used so far in this call
   // timing of one kernel class inside the sampler graph
   int timing = 0;
   std::vector<cudaEvent_t> events;
@@ -239,13 +231,6 @@ struct fh_dit {
 namespace {
 
 size_t elt(const fh_dit* m) { return m->bf16 ? 2 : 4; }
-
-// whether any of the block's GEMMs runs on CTA pairs (and so needs the stream-K buffers)
-bool uses_pair_gemms(const fh_dit* m) {
-  if (!m->bf16) return false;
-  const int D = m->D, FF = m->FF;
-  return tile_cfg(3 * D, D).pair || tile_cfg(D, D).pair || tile_cfg(FF, D).pair || tile_cfg(D, FF).pair;
-}
 
 WsLayout layout(const fh_dit* m, int B) {
   WsLayout w{};
@@ -293,28 +278,8 @@ WsLayout layout(const fh_dit* m, int B) {
     w.au_h2 = take(R * HID * 4);
     w.au_tok = take(R * TN * 4);
   }
-  // stream-K partial sums of the CTA-pair GEMMs: one slot of 2 x 128 rows x 256 fp32 per
-  // cluster (one per CTA pair of the GPU), and per-(tile, CTA, 32-row quarter) counters
-  // and one counter per launch of the gated-residual GEMM that normalises the rows it finished
-  // (LN_COUNTERS per call); counters and flags sit together and start every call at zero
-  w.sk_part = w.sk_flags = w.sk_flags_bytes = w.ln_ctr = 0;
-  if (uses_pair_gemms(m)) {
-    const size_t tiles = ((M + 255) / 256) * (size_t)((std::max(3 * m->D, m->FF) + 127) / 128);
-    w.sk_part = take((size_t)(m->num_sms / 2) * 2 * 128 * 256 * 4);
-    const size_t flags = al256(tiles * 2 * 4 * 4);
-    w.sk_flags = take(flags + LN_COUNTERS * 4);
-    w.ln_ctr = w.sk_flags + flags;
-    w.sk_flags_bytes = flags + LN_COUNTERS * 4;
-  }
   w.total = o;
   return w;
-}
-
-// the stream-K flags and the norm counters start every call at zero (stream-K owners also
-// clear their flags as they go)
-cudaError_t clear_sk_flags(const WsLayout& w, void* ws, cudaStream_t st) {
-  if (!w.sk_flags_bytes) return cudaSuccess;
-  return cudaMemsetAsync(reinterpret_cast<uint8_t*>(ws) + w.sk_flags, 0, w.sk_flags_bytes, st);
 }
 
 template <typename P>
@@ -348,10 +313,6 @@ int get_plan(fh_dit* m, void* ws, int B, Plan** out) {
     ok = ok && make_map_3d(&p.m_xq, at<void>(ws, w.cq), m->D, HW, frames, 64, 128) &&
          make_map_3d(&p.m_xo, at<void>(ws, w.attn), m->D, HW, frames, 64, 32) &&
          make_map(&p.m_xkv, at<void>(ws, w.ckv), frames * m->A, (uint64_t)m->NB * 2 * m->D, 32);
-    if (ok && w.sk_flags_bytes) {
-      const uint64_t rows = (uint64_t)(m->num_sms / 2) * 256;
-      ok = make_out_map(&p.m_skp, at<void>(ws, w.sk_part), rows, 256, 256, true);
-    }
     if (!ok) {
       p.ws = nullptr;
       return fail(FH_ERR_CUDA, "tensor map encoding failed for the workspace");
@@ -376,19 +337,9 @@ void timed_end(fh_dit* m, int i, cudaStream_t st) {
   m->last_pairs.push_back(i);
 }
 
-// The norm a gated-residual GEMM may apply to the rows it finished (rownorm.cuh): mode, the
-// scale / weight vector a, the shift / bias vector c, and a's and c's stride per stream.
-struct NormSpec {
-  int mode;
-  const float* a;
-  const float* c;
-  long bstride;
-};
-
 int run_gemm(fh_dit* m, const CUtensorMap* amap, const void* A, long lda, const CUtensorMap* bmap, const void* W,
              long ldw, int M, int N, int K, int kind, bool out_bf16, const EpiParams& ep, cudaStream_t st,
-             int tclass, const NormSpec* norm = nullptr, void* norm_out = nullptr, bool* normed = nullptr) {
-  if (normed) *normed = false;
+             int tclass) {
   const int ti = timed_begin(m, tclass, st);
   cudaError_t e;
   if (m->bf16) {
@@ -398,32 +349,12 @@ int run_gemm(fh_dit* m, const CUtensorMap* amap, const void* A, long lda, const 
       timed_end(m, ti, st);
       return fail(FH_ERR_CUDA, "tensor map encoding failed for a GEMM output");
     }
-    EpiParams epk = ep;
-    const WsLayout& w = m->plan.lay;
-    const bool sk = tc.pair && tc.streamk && w.sk_flags_bytes;
-    if (sk) {  // stream-K over every CTA pair
-      epk.sk_part = at<float>(m->plan.ws, w.sk_part);
-      epk.sk_flags = at<int>(m->plan.ws, w.sk_flags);
-    }
-    if (tc.pair && w.sk_flags_bytes) {
-      // the next norm of the updated rows, in the same launch (width 1536, a counter left)
-      if (kFuseNorms && norm && kind == EPI_RESID && N == 12 * 128 && m->ln_seq < LN_COUNTERS) {
-        epk.ln_out = norm_out;
-        epk.ln_mode = norm->mode;
-        epk.ln_a = norm->a;
-        epk.ln_c = norm->c;
-        epk.ln_bstride = norm->bstride;
-        epk.ln_eps = m->cfg.eps;
-        epk.ln_ctr = at<int>(m->plan.ws, w.ln_ctr) + m->ln_seq++;
-        if (normed) *normed = true;
-      }
-    }
-    e = gemm_tc(*amap, *bmap, tc.pair ? &cmap : nullptr, sk ? &m->plan.m_skp : nullptr, M, N, K, tc.bn, kind,
-                out_bf16, epk, m->err_dev, m->num_sms, st, tc.pair);
-  }
-  else
+    e = gemm_tc(*amap, *bmap, tc.pair ? &cmap : nullptr, M, N, K, tc.bn, kind, out_bf16, ep, m->err_dev,
+                m->num_sms, st, tc.pair);
+  } else {
     e = gemm_simt(reinterpret_cast<const float*>(A), lda, reinterpret_cast<const float*>(W), ldw, M, N, K, kind,
                   ep, st);
+  }
   timed_end(m, ti, st);
   m->launches++;
   if (e != cudaSuccess) return fail(FH_ERR_CUDA, "gemm launch (M=%d N=%d K=%d kind=%d): %s", M, N, K, kind,
@@ -499,13 +430,9 @@ int run_cross_kv(fh_dit* m, Plan& P, int k0, int nb, cudaStream_t st) {
                   m->bf16, ep, st, 0);
 }
 
-// One block on the residual x. h_ready: the block's first norm (LN1 and its modulation) is
-// already in h (the previous block's FFN2 wrote it). after: the norm that follows the block
-// (the next block's LN1, or the output norm), which the block's last GEMM applies to the rows
-// it finishes when it can; *after_done says whether it did.
+// One block on the residual x.
 template <typename T>
-int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec* after, bool* after_done,
-              cudaStream_t st) {
+int run_block(fh_dit* m, Plan& P, int k, float* x, cudaStream_t st) {
   const WsLayout& w = P.lay;
   void* ws = P.ws;
   const int B = P.batch, L = m->L, D = m->D, NH = m->NH;
@@ -518,10 +445,9 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec*
   T* qkv = at<T>(ws, w.qkv);
   float* ssq_qk = at<float>(ws, w.ssq_qk);
   const float eps = m->cfg.eps;
-  if (after_done) *after_done = false;
 
   // self-attention branch
-  if (!h_ready) {
+  {
     const int ti = timed_begin(m, 6, st);
     cudaError_t e = norm_rows<T>(x, h, M, D, L, 0, mods + 0 * D, mods + 1 * D, mbs, nullptr, nullptr, eps, st);
     timed_end(m, ti, st);
@@ -552,7 +478,6 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec*
     timed_end(m, ti, st);
     LAUNCH(e);
   }
-  bool normed = false;
   {
     // O-proj + gated residual, then the learned-affine LayerNorm before the cross-attention (R7)
     EpiParams ep = epi0(L);
@@ -561,12 +486,10 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec*
     ep.ldr = D;
     ep.gate = mods + 2 * D;
     ep.gate_bstride = mbs;
-    const NormSpec ln3{1, bw.ln3w, bw.ln3b, 0};
-    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_o, bw.wo, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1, &ln3, h,
-                 &normed));
+    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_o, bw.wo, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1));
   }
   // audio cross-attention branch
-  if (!normed) LAUNCH(norm_rows<T>(x, h, M, D, L, 1, nullptr, nullptr, 0, bw.ln3w, bw.ln3b, eps, st));
+  LAUNCH(norm_rows<T>(x, h, M, D, L, 1, nullptr, nullptr, 0, bw.ln3w, bw.ln3b, eps, st));
   {
     EpiParams ep = epi0(L);
     ep.bias = bw.bcq;
@@ -597,12 +520,10 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec*
     ep.bias = bw.bco;
     ep.resid = x;
     ep.ldr = D;
-    const NormSpec ln2{0, mods + 4 * D, mods + 3 * D, mbs};
-    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_co, bw.wco, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1, &ln2, h,
-                 &normed));
+    RUN(run_gemm(m, &P.m_attn, attn, D, &bw.m_co, bw.wco, D, M, D, D, EPI_RESID, m->bf16, ep, st, 1));
   }
   // FFN branch
-  if (!normed) LAUNCH(norm_rows<T>(x, h, M, D, L, 0, mods + 3 * D, mods + 4 * D, mbs, nullptr, nullptr, eps, st));
+  LAUNCH(norm_rows<T>(x, h, M, D, L, 0, mods + 3 * D, mods + 4 * D, mbs, nullptr, nullptr, eps, st));
   {
     EpiParams ep = epi0(L);
     ep.bias = bw.b1;
@@ -618,7 +539,7 @@ int run_block(fh_dit* m, Plan& P, int k, float* x, bool h_ready, const NormSpec*
     ep.gate = mods + 5 * D;
     ep.gate_bstride = mbs;
     RUN(run_gemm(m, &P.m_u, at<T>(ws, w.u), m->FF, &bw.m_2, bw.w2, m->FF, M, D, m->FF, EPI_RESID, m->bf16, ep, st,
-                 1, after, h, after_done));
+                 1));
   }
   return FH_OK;
 }
@@ -640,16 +561,9 @@ int run_network(fh_dit* m, Plan& P, cudaStream_t st) {
                  false, ep, st, 0));
   }
   float* hm = at<float>(ws, w.hmods);
-  const long mbs = (long)m->NB * 6 * D;
-  bool h_ready = false;
-  for (int k = 0; k < m->NB; ++k) {
-    // after block k: the next block's LN1 with its modulation, or the output RMSNorm (R9)
-    const float* nm = at<float>(ws, w.mods) + (long)(k + 1) * 6 * D;
-    const NormSpec next = k + 1 < m->NB ? NormSpec{0, nm + D, nm, mbs} : NormSpec{2, hm + D, hm, 2L * D};
-    RUN(run_block<T>(m, P, k, x, h_ready, &next, &h_ready, st));
-  }
-  if (!h_ready)
-    LAUNCH(norm_rows<T>(x, at<T>(ws, w.h), M, D, L, 2, hm, hm + D, 2L * D, nullptr, nullptr, m->cfg.eps, st));
+  for (int k = 0; k < m->NB; ++k) RUN(run_block<T>(m, P, k, x, st));
+  // the output norm with its modulation (R9)
+  LAUNCH(norm_rows<T>(x, at<T>(ws, w.h), M, D, L, 2, hm, hm + D, 2L * D, nullptr, nullptr, m->cfg.eps, st));
   {
     EpiParams ep = epi0(L);
     ep.bias = m->head_b;
@@ -1008,9 +922,7 @@ int fh_dit_block_forward(fh_dit* m, int block, const float* x_in, float* x_out, 
   Plan* P;
   RUN(get_plan(m, ws, batch, &P));
   m->launches = 0;
-  m->ln_seq = 0;
   const size_t M = (size_t)batch * m->L;
-  CK(clear_sk_flags(P->lay, ws, st));
   CK(cudaMemcpyAsync(at<void>(ws, P->lay.audio), audio, (size_t)batch * m->F * m->A * m->D * elt(m),
                      cudaMemcpyDeviceToDevice, st));
   if (x_out != x_in) CK(cudaMemcpyAsync(x_out, x_in, M * m->D * 4, cudaMemcpyDeviceToDevice, st));
@@ -1019,9 +931,9 @@ int fh_dit_block_forward(fh_dit* m, int block, const float* x_in, float* x_out, 
   RUN(run_cross_kv(m, *P, block, 1, st));
   RUN(run_time_cond(m, *P, tv, st));
   if (m->bf16)
-    RUN(run_block<bf16>(m, *P, block, x_out, false, nullptr, nullptr, st));
+    RUN(run_block<bf16>(m, *P, block, x_out, st));
   else
-    RUN(run_block<float>(m, *P, block, x_out, false, nullptr, nullptr, st));
+    RUN(run_block<float>(m, *P, block, x_out, st));
   m->last_launches = m->launches;
   return FH_OK;
 }
@@ -1036,9 +948,7 @@ int fh_dit_predict_flow(fh_dit* m, const float* x_noisy, const float* ref, const
   Plan* P;
   RUN(get_plan(m, ws, batch, &P));
   m->launches = 0;
-  m->ln_seq = 0;
   const WsLayout& w = P->lay;
-  CK(clear_sk_flags(w, ws, st));
   CK(cudaMemcpyAsync(at<void>(ws, w.audio), audio, (size_t)batch * m->F * m->A * m->D * elt(m),
                      cudaMemcpyDeviceToDevice, st));
   TVals tv;
@@ -1085,7 +995,6 @@ static int sample_impl(fh_dit* m, const float* noise, const float* ref, const fl
     CK(cudaStreamBeginCapture(m->cap, cudaStreamCaptureModeRelaxed));
     m->capturing = true;
     m->launches = 0;
-    m->ln_seq = 0;
     m->ev_used = 0;
     m->last_pairs.clear();
     int rc = m->bf16 ? run_sampler_steps<bf16>(m, *P, sigmas, nsteps, eps, m->cap)
@@ -1115,7 +1024,6 @@ static int sample_impl(fh_dit* m, const float* noise, const float* ref, const fl
     m->graphs.push_back(ge);
     g = &m->graphs.back();
   }
-  CK(clear_sk_flags(w, ws, st));
   CK(cudaGraphLaunch(g->exec, st));
   m->last_pairs = g->ev_pairs;
   m->launches = outside + g->launches;
@@ -1323,55 +1231,13 @@ int fh_op_linear(const void* A, const void* W, const float* bias, float* out, in
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     RUN(prepare_device(dev));
-    e = gemm_tc(ma, mb, &mc, nullptr, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, tc.pair);
+    e = gemm_tc(ma, mb, &mc, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, tc.pair);
   } else if (dtype == FH_F32) {
     if (K % 32) return fail(FH_ERR_SHAPE, "K %% 32 != 0");
     e = gemm_simt((const float*)A, K, (const float*)W, K, M, N, K, EPI_STORE, ep, st);
   } else {
     return fail(FH_ERR_ARG, "bad dtype");
   }
-  if (e != cudaSuccess) return fail(FH_ERR_CUDA, "linear launch: %s", cudaGetErrorString(e));
-  return FH_OK;
-}
-
-size_t fh_op_linear_streamk_bytes(int M, int N, int K) {
-  if (M < 1 || N < 128 || N % 128 || K < 64 || K % 64) return 0;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const size_t tiles = ((size_t)(M + 255) / 256) * (size_t)(N / 128);
-  return al256((size_t)(sms / 2) * 256 * 256 * 4) + al256(tiles * 8 * 4);
-}
-
-int fh_op_linear_streamk(const void* A, const void* W, const float* bias, float* out, int M, int N, int K, void* ws,
-                         size_t ws_bytes, void* stream) {
-  if (!A || !W || !bias || !out || !ws || !aligned16(A) || !aligned16(W) || !aligned16(bias) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(ws) & 255))
-    return fail(FH_ERR_ARG, "null or unaligned pointer");
-  if (M < 1 || N % 128 || K % 64) return fail(FH_ERR_SHAPE, "bad GEMM shape %d x %d x %d", M, N, K);
-  const TileCfg tc = tile_cfg(N, K);
-  if (!tc.pair) return fail(FH_ERR_SHAPE, "shape %d x %d x %d does not run on CTA pairs", M, N, K);
-  const size_t need = fh_op_linear_streamk_bytes(M, N, K);
-  if (ws_bytes < need) return fail(FH_ERR_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
-  if (!load_encode()) return fail(FH_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled unavailable");
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  RUN(prepare_device(dev));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t part_bytes = al256((size_t)(sms / 2) * 256 * 256 * 4);
-  EpiParams ep = epi0(1 << 30);
-  ep.bias = bias;
-  ep.out = out;
-  ep.ldo = N;
-  ep.sk_part = reinterpret_cast<float*>(ws);
-  ep.sk_flags = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ws) + part_bytes);
-  CUtensorMap ma, mb, mc, mp;
-  if (!make_map(&ma, A, M, K, 128) || !make_map(&mb, W, N, K, tc.wbox) || !make_out_map(&mc, out, M, N, N, true) ||
-      !make_out_map(&mp, ws, (uint64_t)(sms / 2) * 256, 256, 256, true))
-    return fail(FH_ERR_CUDA, "tensor map encoding");
-  CK(cudaMemsetAsync(ep.sk_flags, 0, need - part_bytes, st));
-  const cudaError_t e = gemm_tc(ma, mb, &mc, &mp, M, N, K, tc.bn, EPI_STORE, false, ep, nullptr, sms, st, true);
   if (e != cudaSuccess) return fail(FH_ERR_CUDA, "linear launch: %s", cudaGetErrorString(e));
   return FH_OK;
 }

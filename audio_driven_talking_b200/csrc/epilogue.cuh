@@ -45,22 +45,6 @@ struct EpiParams {
   const float2* rope;     // EPI_QKV: (cos, sin) [rows_per_batch, 64]
   int dim;                // EPI_QKV: width D of each of the q, k, v sections
   long sec_stride;        // EPI_QKV: elements per section = B * heads * L * 128
-  // CTA-pair GEMM, stream-K: fp32 partial sums [clusters][2][128][BN] and per-(tile, CTA,
-  // 32-row quarter) counters (zero between launches); null sk_part: whole tiles per cluster
-  float* sk_part;
-  int* sk_flags;
-  // EPI_RESID on CTA pairs (width 1536): once every CTA of the launch has added its tiles to
-  // the residual, the CTAs normalise its rows for the next step (rownorm.cuh, mode ln_mode)
-  // into ln_out [M, N] bf16; ln_a / ln_c are the scale / shift (modes 0, 2; stride
-  // ln_bstride per stream) or weight / bias (mode 1) vectors; ln_ctr a counter, zero on entry,
-  // that no other launch uses. ln_out null: no norm.
-  void* ln_out;
-  int ln_mode;
-  const float* ln_a;
-  const float* ln_c;
-  long ln_bstride;
-  float ln_eps;
-  int* ln_ctr;
 };
 
 __device__ __forceinline__ bool epi_normed(const EpiParams& p, int col) {

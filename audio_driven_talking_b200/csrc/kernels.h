@@ -40,13 +40,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // two CTAs of a cluster with cta_group::2, persistent over every CTA pair; their epilogues
 // store through `c`, a TMA map of the output (EPI_RESID: of the fp32 residual; EPI_QKV: 3D
 // [3*B*heads][L][128]) with box 32 x 32 (x 1) and the 128-byte (fp32) or 64-byte (bf16)
-// swizzle. With ep.sk_part set the pairs split the k-blocks stream-K: `p` is then a 2D fp32
-// map of the partial-sum slots [pairs * 256 rows][256] with box 32 x 32 and the 128-byte
-// swizzle, and ep.sk_flags the per-(tile, CTA, quarter) counters, zero on entry.
+// swizzle.
 cudaError_t gemm_tc_prepare();  // sets the kernels' shared-memory attributes on the current device
-cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, const CUtensorMap* p, int M,
-                    int N, int K, int bn, int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms,
-                    cudaStream_t st, bool pair = false);
+cudaError_t gemm_tc(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap* c, int M, int N, int K, int bn,
+                    int kind, bool out_bf16, const EpiParams& ep, unsigned* err, int num_sms, cudaStream_t st,
+                    bool pair = false);
 
 // fp32 CUDA-core GEMM (misc.cu) with the same epilogues; N % 128 == 0.
 cudaError_t gemm_simt(const float* A, long lda, const float* W, long ldw, int M, int N, int K, int kind,

@@ -23,19 +23,6 @@ extern "C" {
 int fh_op_linear(const void* A, const void* W, const float* bias, float* out, int M, int N, int K, int dtype,
                  void* stream);
 
-/* fh_op_linear (dtype FH_BF16) on 256-row CTA-pair tiles with the k-blocks of all tiles
- * split evenly over every CTA pair of the GPU (stream-K), the way the model's block
- * projections run: a tile cut between pairs is finished by the pair holding its first
- * k-blocks, which adds the others' fp32 partial sums in k order (deterministic). Only for
- * shapes that run on CTA pairs (K >= 1024, 1536 <= N <= 16384, N % 128 == 0, K % 64 == 0;
- * else FH_ERR_SHAPE). ws: caller-owned device scratch, 256-byte aligned, of at least
- * fh_op_linear_streamk_bytes(M, N, K) bytes (else FH_ERR_ARG; the call clears the part that
- * must start at zero); calls sharing a ws must not overlap in time.
- * fh_op_linear_streamk_bytes returns 0 for an invalid shape. */
-size_t fh_op_linear_streamk_bytes(int M, int N, int K);
-int fh_op_linear_streamk(const void* A, const void* W, const float* bias, float* out, int M, int N, int K, void* ws,
-                         size_t ws_bytes, void* stream);
-
 /* Non-causal self-attention over L tokens per (stream, head), as inside a block
  * (gizai:flashhead, opening paragraph; readings R4-R6): q, k, v [batch, heads, L,
  * 128] in dtype, except that with FH_BF16 v is float16 (as the QKV projection stores it:

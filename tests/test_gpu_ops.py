@@ -42,14 +42,14 @@ def test_linear_bf16_tensor_core(M, N, K):
 @pytest.mark.parametrize("M,N,K", [(1280, 1536, 1536), (1280, 4608, 1536), (1280, 1536, 8960), (1280, 8960, 1536),
                                    (8640, 8960, 1536), (8640, 1536, 8960), (520, 1536, 1536), (300, 1536, 1024),
                                    (4000, 1536, 4096), (256, 1536, 1024), (864, 4608, 1536)])
-def test_linear_bf16_stream_k(M, N, K):
-    """CTA-pair tiles with the k-blocks split evenly over all CTA pairs: tiles cut between
-    pairs (two, three or more pieces) are summed by their owner; repeated calls agree
-    bitwise (the partial sums are added in a fixed order)."""
+def test_linear_bf16_pair_tiles(M, N, K):
+    """The CTA-pair GEMMs at the model's projection shapes and ragged row counts: persistent
+    pairs with several tiles each, the split-K clusters of four (N = 1536), the last rows of a
+    ragged tile; repeated calls agree bitwise."""
     A, W, b = _bf16_operands(M * 3 + N + K, M, N, K)
     Ad, Wd, bd = to_dev(A, torch.bfloat16), to_dev(W, torch.bfloat16), to_dev(b)
-    out = fh.linear_streamk(Ad, Wd, bd)
-    out2 = fh.linear_streamk(Ad, Wd, bd)
+    out = fh.linear(Ad, Wd, bd)
+    out2 = fh.linear(Ad, Wd, bd)
     torch.cuda.synchronize()
     assert torch.equal(out, out2)
     rows = np.unique(np.concatenate([np.arange(0, M, max(1, M // 512)), np.arange(max(0, M - 40), M)]))
