@@ -134,10 +134,11 @@ struct TileCfg {
 TileCfg tile_cfg(int N, int K, bool pair_ok = true) {
   TileCfg t;
   t.pair = pair_ok && K >= 1024 && N >= 1536 && N <= 16384;
-  // 256 wide for the cross-KV (single CTAs) and for the pair GEMMs of width up to 4096
+  // 256 wide for the cross-KV (single CTAs), for QKV (N = 4608: the pair's operand bytes per
+  // MMA, not its MMA rate, bound these main loops) and for the pair GEMMs of width up to 4096
   // (O-proj, cross-Q/O, FFN2), which then run split-K on clusters of four when their 256 x 256
-  // tiles are few; 128 for QKV
-  t.bn = (N % 256 == 0 && (N >= 8192 || (t.pair && N <= 4096))) ? 256 : 128;
+  // tiles are few
+  t.bn = (N % 256 == 0 && (N >= 4608 || (t.pair && N <= 4096))) ? 256 : 128;
   // FFN1 (N = 8960 = 40 x 224): at 1280 tokens 200 pair tiles of width 224 fill three rounds
   // of 74 CTA pairs better than 175 tiles of width 256
   if (t.pair && N >= 8192 && N % 224 == 0) t.bn = 224;

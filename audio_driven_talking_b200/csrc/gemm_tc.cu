@@ -304,8 +304,10 @@ struct Tc2Shape {
   static constexpr uint32_t TX_BYTES = 2 * STAGE_BYTES;  // both CTAs' loads complete on the even CTA's barrier
   // two accumulators of BN columns, allocated as a power of two
   static constexpr uint32_t TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-  // epilogue staging: per epilogue warp two 32-row boxes of up to 128-byte rows
-  static constexpr uint32_t STG_BYTES = EPI_WARPS * 2 * 4096;
+  // epilogue staging: per epilogue warp STG_BOXES 32-row boxes of up to 128-byte rows (one:
+  // the ring's bytes in flight, not the epilogue, bound these main loops)
+  static constexpr int STG_BOXES = 1;
+  static constexpr uint32_t STG_BYTES = EPI_WARPS * STG_BOXES * 4096;
   static constexpr uint32_t AUX_BYTES = 2048;  // barriers and the norm hand-over
   // the operand ring takes what is left of the 227 KB a CTA may use (up to 8 stages)
   static constexpr int FIT = (int)((227u * 1024u - 1024u - AUX_BYTES - STG_BYTES) / STAGE_BYTES);
@@ -475,7 +477,7 @@ __global__ void __launch_bounds__(TC2_THREADS, 1)
     const int sub = (warp - 2) >> 2;  // 0: columns [0, EPI_SPLIT), 1: [EPI_SPLIT, BN)
     const int cbeg = sub ? S::EPI_SPLIT : 0;
     const int cend = sub ? BN : S::EPI_SPLIT;
-    uint8_t* stg = smem + S::RING_BYTES + (warp - 2) * 8192;  // this warp's two staging boxes
+    uint8_t* stg = smem + S::RING_BYTES + (warp - 2) * (S::STG_BOXES * 4096);  // this warp's staging boxes
     uint32_t nchunk = 0;
     uint32_t nx = 0;  // norm hand-overs between this quarter's two warps so far
     pdl_wait();
@@ -523,9 +525,9 @@ __global__ void __launch_bounds__(TC2_THREADS, 1)
             for (int j = 0; j < 32; ++j) v[j] = 0.f;
           }
           // buffers alternate per committed store, so the one group that may still be
-          // reading is the other buffer's
-          uint8_t* box = stg + (nchunk & 1) * 4096;
-          if (lane == 0) bulk_wait_read<1>();
+          // reading is the other buffer's (one buffer: no group may still be reading it)
+          uint8_t* box = stg + (S::STG_BOXES == 2 ? (nchunk & 1) * 4096 : 0);
+          if (lane == 0) bulk_wait_read<S::STG_BOXES - 1>();
           __syncwarp();
           if (KIND == EPI_QKV && std::is_same<OutT, bf16>::value && (n0 + c) / ep.dim == 2)
             stage_row(box, lane, v, (__half*)nullptr);  // v in fp16 (epilogue.cuh, EPI_QKV)
