@@ -64,10 +64,7 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ float row_rms(const float* ssq, int ssq_ld, long row, int off, int heads, float inv_d,
                                          float eps) {
-  const float* p = ssq + row * ssq_ld + off;
-  float s = 0.f;
-  for (int h = 0; h < heads; ++h) s += p[h];
-  return rsqrtf(s * inv_d + eps);
+  return rsqrtf(sum_heads(ssq + row * ssq_ld + off, heads) * inv_d + eps);
 }
 
 // Every key's RMS factor rk[key] (0 past L) for keys [0, nkeys), by `nthreads` threads: with
@@ -123,9 +120,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
   // tiles back is always complete (S_j waits for P_{j-2} V_{j-2}) and the one two tiles
   // ahead cannot start, so each wait names one phase.
   uint64_t* pv_done = bars + 15;
-  uint64_t* rk_full = bars + 19;  // every key's RMS factor staged
+  uint64_t* rk_full = bars + 19;  // the first key RMS factors staged
   uint64_t* fin_bar = bars + 20;  // both halves' (m, l) published
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 21);
+  uint64_t* rk_bar = bars + 21;   // [2 halves][2 tiles by parity] a later tile's key RMS factors staged
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 25);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -150,6 +148,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     }
     mbar_init(rk_full, AT_SOFTMAX_THREADS);
     mbar_init(fin_bar, AT_SOFTMAX_THREADS);
+    for (int i = 0; i < 4; ++i) mbar_init(&rk_bar[i], AT_SOFTMAX_THREADS / 2);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tmQ);
@@ -294,16 +293,37 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
     const int qi = qt * AT_BQ + rl;                    // query index within the stream
     const bool qvalid = qi < L;
     const float inv_d = 1.f / (float)D;
-    const float rq = row_rms(ssq, ssq_ld, (long)b * L + (qvalid ? qi : L - 1), 0, heads, inv_d, eps);
-    const float qscale = rq * scale_log2;
+    // the query's own partial sums, loaded now and added after the keys' loads are issued, so
+    // that the prologue waits for one round trip to L2, not two
+    const float* qrow = ssq + ((long)b * L + (qvalid ? qi : L - 1)) * ssq_ld;
+    const bool qvec = heads == 12 && (reinterpret_cast<uintptr_t>(qrow) & 15) == 0;
+    float4 qv[3];
+    if (qvec) {
+#pragma unroll
+      for (int c = 0; c < 3; ++c) qv[c] = reinterpret_cast<const float4*>(qrow)[c];
+    }
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t o_t = tmem + lane_off + 256 + half * 128;  // this half's O accumulator row
     float* mls = reinterpret_cast<float*>(smem + OFF_ML);    // [2 halves][m, l][128 rows]
 
-    // every key's RMS factor, once per CTA (the keys are shared by all tiles of the row)
+    // The keys' RMS factors, staged in shared memory (every row of the tile uses them). With
+    // 12 heads only the first two tiles' are computed before the loop; each later tile's are
+    // loaded by its half's threads two tiles ahead (one key per thread, three 16-byte loads
+    // issued at the start of a tile and summed at its end, so their L2 latency hides behind
+    // the exponentials). Otherwise every key's, before the loop.
     float* rk_all = reinterpret_cast<float*>(smem + OFF_RKALL);
-    key_rms_all(rk_all, ssq, ssq_ld, (long)b * L, heads, L, nkv * AT_BK, inv_d, eps, t, AT_SOFTMAX_THREADS);
+    const bool lazy = heads == 12 && (ssq_ld & 3) == 0 && (reinterpret_cast<uintptr_t>(ssq) & 15) == 0;
+    key_rms_all(rk_all, ssq, ssq_ld, (long)b * L, heads, L, (lazy && nkv > 2 ? 2 : nkv) * AT_BK, inv_d, eps, t,
+                AT_SOFTMAX_THREADS);
     mbar_arrive(rk_full);
+    float qs = 0.f;  // head by head in order, as sum_heads adds them
+    if (qvec) {
+#pragma unroll
+      for (int c = 0; c < 3; ++c) qs = (((qs + qv[c].x) + qv[c].y) + qv[c].z) + qv[c].w;
+    } else {
+      qs = sum_heads(qrow, heads);
+    }
+    const float qscale = rsqrtf(qs * inv_d + eps) * scale_log2;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = mbar_wait(rk_full, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
     ok = __all_sync(0xffffffffu, ok);
@@ -311,6 +331,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       const float* rk = rk_all + j * AT_BK + half * 64;
       const int bf = j & 1;
       ok = mbar_wait(&s_full[bf], (j >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
+      // tile j + 2's key factors (this half's 64 keys, one per thread of its first 64)
+      float4 kp[3];
+      const int kkey = (lazy && j + 2 < nkv && (t & 127) < 64) ? (j + 2) * AT_BK + half * 64 + (t & 127) : -1;
+      if (kkey >= 0) {
+        const float4* p = reinterpret_cast<const float4*>(ssq + ((long)b * L + (kkey < L ? kkey : 0)) * ssq_ld + heads);
+#pragma unroll
+        for (int c = 0; c < 3; ++c) kp[c] = p[c];
+      }
+      // this tile's key factors, staged two tiles ago
+      if (ok && lazy && j >= 2)
+        ok = mbar_wait(&rk_bar[2 * half + (j & 1)], ((j - 2) >> 1) & 1, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -398,6 +429,15 @@ __global__ void __launch_bounds__(AT_THREADS, 1)
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[2 * half + bf]);
+      if (lazy && j + 2 < nkv) {
+        if (kkey >= 0) {
+          float s2 = 0.f;
+#pragma unroll
+          for (int c = 0; c < 3; ++c) s2 += (kp[c].x + kp[c].y) + (kp[c].z + kp[c].w);
+          rk_all[kkey] = kkey < L ? rsqrtf(s2 * inv_d + eps) : 0.f;
+        }
+        mbar_arrive(&rk_bar[2 * half + (j & 1)]);
+      }
     }
     if (ok) {
       // this half's last product, then both halves' (m, l) for the combination

@@ -35,6 +35,23 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Sum of one row's per-head partial sums of squares (p: the row's first head), added head by
+// head in order: with the model's 12 heads the values arrive by three 16-byte loads in flight
+// at once, not a chain of dependent ones.
+__device__ __forceinline__ float sum_heads(const float* p, int heads) {
+  float s = 0.f;
+  if (heads == 12 && (reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    float4 v[3];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) v[c] = reinterpret_cast<const float4*>(p)[c];
+#pragma unroll
+    for (int c = 0; c < 3; ++c) s = (((s + v[c].x) + v[c].y) + v[c].z) + v[c].w;
+  } else {
+    for (int h = 0; h < heads; ++h) s += p[h];
+  }
+  return s;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -1,5 +1,4 @@
-// rownorm.cuh - one row's norm and modulation, by one warp (shared by the row-norm kernel and
-// the gated-residual GEMM, which can normalise the rows it has just finished).
+// rownorm.cuh - one row's norm and modulation, by one warp.
 //
 // D = 128 * NV floats held in registers (a float4 per lane per step). Mode 0 / 2: the adaLN
 // modulate h = n(x) * (1 + scale) + shift of the Wan-style block (reading R1) and of the

@@ -111,10 +111,7 @@ __global__ void __launch_bounds__(XT_THREADS, 1)
       tma_load_2d(&tmKV, kv_full, smem + XT_OFF_V + XT_PANEL_KV, voff + h * 128 + 64, (int)kv_row0);
     }
     // key `lane`'s RMS factor over the full width (all heads' partial sums)
-    const float* p = ssq_k + (kv_row0 + lane) * ssq_k_ld + ssq_k_off;
-    float s = 0.f;
-    for (int i = 0; i < heads; ++i) s += p[i];
-    rks[lane] = rsqrtf(s * inv_d + eps);
+    rks[lane] = rsqrtf(sum_heads(ssq_k + (kv_row0 + lane) * ssq_k_ld + ssq_k_off, heads) * inv_d + eps);
     mbar_arrive(rk_full);
     if (lane == 0) {
       // the CTA's shared memory must outlive the copies: wait for them whatever happened
@@ -161,10 +158,7 @@ __global__ void __launch_bounds__(XT_THREADS, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     float rq = 1.f;
     if (valid) {
-      const float* p = ssq_q + ((long)frame * HW + n) * heads;
-      float s = 0.f;
-      for (int i = 0; i < heads; ++i) s += p[i];
-      rq = rsqrtf(s * inv_d + eps);
+      rq = rsqrtf(sum_heads(ssq_q + ((long)frame * HW + n) * heads, heads) * inv_d + eps);
     }
     const float qscale = rq * scale_log2;
     bool ok = mbar_wait(rk_full, 0, abort_flag, err, ERRBIT_TIMEOUT_ATTN);
