@@ -182,10 +182,25 @@ __global__ void time_sinusoid_kernel(float* out, int batch, TVals tv, int dim) {
 }
 
 // y[b, n] = act(sum_k W[n, k] * act_in(x[b, k]) + bias[n]); one warp per output.
+constexpr int GV_CHUNKS = 8;  // 16-byte bf16 loads per lane held in registers (K up to 2048)
 template <typename WT>
 __global__ void gemv_kernel(const WT* __restrict__ W, const float* __restrict__ x, const float* __restrict__ bias,
                             float* __restrict__ y, int N, int K, int batch, int silu_in, int silu_out) {
   pdl_launch_dependents();
+  const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const WT* wr = W + (long)(n < N ? n : 0) * K;
+  // bf16 rows: the whole row's weights (8 per lane per 16-byte load) are requested at once,
+  // before the dependency wait (the weights are never written by any kernel), so the loads
+  // overlap the preceding kernel and the staging of x
+  const bool vec = sizeof(WT) == 2 && K % 256 == 0 && K <= 256 * GV_CHUNKS;
+  const int nc = K / 256;
+  uint4 wq[GV_CHUNKS];
+  if (vec) {
+#pragma unroll
+    for (int c = 0; c < GV_CHUNKS; ++c)
+      if (c < nc) wq[c] = __ldg(reinterpret_cast<const uint4*>(wr + c * 256 + lane * 8));
+  }
   pdl_wait();
   extern __shared__ float xs[];
   for (int i = threadIdx.x; i < batch * K; i += blockDim.x) {
@@ -193,18 +208,22 @@ __global__ void gemv_kernel(const WT* __restrict__ W, const float* __restrict__ 
     xs[i] = silu_in ? silu(v) : v;
   }
   __syncthreads();
-  const int n = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
   if (n >= N) return;
   float acc[8];
   for (int b = 0; b < batch; ++b) acc[b] = 0.f;
-  const WT* wr = W + (long)n * K;
-  if (sizeof(WT) == 2 && K % 256 == 0) {
-    // bf16 rows: 16-byte loads, 8 weights per lane per load, two loads in flight
-#pragma unroll 2
-    for (int k0 = lane * 8; k0 < K; k0 += 256) {
+  if (vec) {
+#pragma unroll
+    for (int c = 0; c < GV_CHUNKS; ++c) {
+      if (c >= nc) break;
+      const int k0 = c * 256 + lane * 8;
       float w8[8];
-      load8(reinterpret_cast<const bf16*>(wr) + k0, w8);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&wq[c]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        w8[2 * e] = f.x;
+        w8[2 * e + 1] = f.y;
+      }
       for (int b = 0; b < batch; ++b) {
         const float4 x0 = *reinterpret_cast<const float4*>(xs + b * K + k0);
         const float4 x1 = *reinterpret_cast<const float4*>(xs + b * K + k0 + 4);

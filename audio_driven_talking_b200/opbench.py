@@ -6,6 +6,7 @@ for ncu captures of one kernel on a case of a chosen size.
     python -m audio_driven_talking_b200.opbench linear --m 1280 --n 1536 --k 1536
     python -m audio_driven_talking_b200.opbench cross_attention --tokens 1280
     python -m audio_driven_talking_b200.opbench slice --blocks 2 --iters 3 [--renoise]
+    python -m audio_driven_talking_b200.opbench slice_kernels --blocks 30
 
 Each prints one JSON line: the operator, its shape, the average time per launch in
 microseconds (CUDA events on the launching stream, after warm-up launches, synchronised on
@@ -138,9 +139,46 @@ def slice_(a):
     return {"op": "slice", "blocks": a.blocks, "steps": len(sig) - 1, "renoise": bool(a.renoise), "us": us}
 
 
+def slice_kernels(a):
+    """One sampler slice of a model of `blocks` blocks replayed from its CUDA graph under the
+    CUDA profiler (CUPTI): per kernel, the spacing of consecutive kernel ends on the stream,
+    i.e. what each kernel adds to the slice once programmatic launches overlap its prologue
+    with its predecessor. Median and total per kernel name."""
+    import collections
+    import statistics
+    import torch
+    from torch.profiler import ProfilerActivity, profile
+    cfg = fh.LITE.replace(blocks=a.blocks)
+    m = fh.DiT(cfg, 1002)
+    ws = m.workspace(1)
+    g = _gen(5)
+    C, F, H, W, A, D = cfg.latent_ch, cfg.frames, cfg.lat_h, cfg.lat_w, cfg.audio_tokens, cfg.dim
+    noise = torch.randn((1, C, F, H, W), device="cuda", generator=g)
+    ref = torch.randn((1, C, F, H, W), device="cuda", generator=g)
+    motion = torch.randn((1, C, 2, H, W), device="cuda", generator=g)
+    audio = torch.randn((1, F, A, D), device="cuda", generator=g).to(torch.bfloat16)
+    sig = [1.0, 0.75, 0.5, 0.25, 0.0]
+    out = torch.empty_like(noise)
+    run = lambda: m.sample_slice(noise, ref, motion, audio, sig, ws, out=out)
+    us = _time(run, a.iters, a.warmup)
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        run()
+        torch.cuda.synchronize()
+    ks = sorted((e.time_range.start, e.time_range.end, e.name) for e in prof.events()
+                if e.device_type == torch.autograd.DeviceType.CUDA)
+    inc = collections.defaultdict(list)
+    for i in range(1, len(ks)):
+        name = ks[i][2].replace("(anonymous namespace)::", "").replace("fh::", "").replace("void ", "")
+        inc[name.split("(")[0]].append(ks[i][1] - ks[i - 1][1])
+    m.close()
+    per = {n: {"launches": len(v), "median_us": statistics.median(v), "total_us": sum(v)}
+           for n, v in sorted(inc.items(), key=lambda kv: -sum(kv[1]))}
+    return {"op": "slice_kernels", "blocks": a.blocks, "steps": len(sig) - 1, "us": us, "kernels": per}
+
+
 def main(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    p.add_argument("op", choices=["row_norm", "attention", "linear", "cross_attention", "slice"])
+    p.add_argument("op", choices=["row_norm", "attention", "linear", "cross_attention", "slice", "slice_kernels"])
     p.add_argument("--rows", type=int, default=65536)
     p.add_argument("--dim", type=int, default=1536)
     p.add_argument("--mode", type=int, default=0)
@@ -158,11 +196,11 @@ def main(argv=None):
     p.add_argument("--graph", action="store_true", help="replay the launches from a CUDA graph")
     a = p.parse_args(argv)
     global GRAPH
-    GRAPH = a.graph and a.op != "slice"  # the sampler records its own graph
+    GRAPH = a.graph and not a.op.startswith("slice")  # the sampler records its own graph
     import torch
     torch.cuda.set_device(0)
     fn = {"row_norm": row_norm, "attention": attention, "linear": linear, "cross_attention": cross_attention,
-          "slice": slice_}[a.op]
+          "slice": slice_, "slice_kernels": slice_kernels}[a.op]
     r = fn(a)
     r["graph"] = GRAPH
     print(json.dumps(r))
