@@ -176,7 +176,7 @@ def slice_kernels(a):
     return {"op": "slice_kernels", "blocks": a.blocks, "steps": len(sig) - 1, "us": us, "kernels": per}
 
 
-def main(argv=None):
+def parser():
     p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     p.add_argument("op", choices=["row_norm", "attention", "linear", "cross_attention", "slice", "slice_kernels"])
     p.add_argument("--rows", type=int, default=65536)
@@ -194,7 +194,11 @@ def main(argv=None):
     p.add_argument("--iters", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--graph", action="store_true", help="replay the launches from a CUDA graph")
-    a = p.parse_args(argv)
+    return p
+
+
+def main(argv=None):
+    a = parser().parse_args(argv)
     global GRAPH
     GRAPH = a.graph and not a.op.startswith("slice")  # the sampler records its own graph
     import torch

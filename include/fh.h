@@ -112,7 +112,9 @@ typedef struct fh_dit fh_dit;
  * constraints), FH_ERR_UNSUPPORTED (not sm_100), FH_ERR_OOM, FH_ERR_CUDA. */
 int fh_dit_create(const fh_config* cfg, uint64_t seed, void* stream, fh_dit** out);
 
-/* Free everything the model owns. NULL is accepted. */
+/* Free everything the model owns (the counterpart of the pages' model load, gizai:flashhead
+ * Functions > load: a model holds its weights on one GPU until it is dropped). NULL is
+ * accepted; the handle must not be used afterwards. Returns FH_OK. */
 int fh_dit_destroy(fh_dit* m);
 
 /* Bytes of caller-allocated workspace (device, 256-byte aligned) that every
@@ -121,22 +123,32 @@ int fh_dit_destroy(fh_dit* m);
  * handle must not overlap in time on the same workspace. */
 size_t fh_dit_workspace_bytes(const fh_dit* m, int batch);
 
-/* One transformer block k for timesteps t (host float32 [batch], in [0, 1]):
- * x_out = block_k(x_in) with x device float32 [B, L, D] (x_in may equal x_out),
- * audio device [B, F, A, D] in the model dtype. The block's adaLN vectors come
- * from the timestep MLP of t; its cross-attention keys/values from `audio`. */
+/* One transformer block k (gizai:flashhead, opening paragraph: one of the 30 Wan-style
+ * blocks, with self-attention over the whole latent and cross-attention to the audio
+ * tokens; readings R1-R8 fix the block's internal order) for timesteps t (host float32
+ * [batch], in [0, 1]): x_out = block_k(x_in) with x device float32 [B, L, D] (x_in may
+ * equal x_out), audio device [B, F, A, D] in the model dtype. The block's adaLN vectors
+ * come from the timestep MLP of t; its cross-attention keys/values from `audio`. Errors:
+ * FH_ERR_ARG (null or unaligned pointer, workspace null or not 256-byte aligned, block out
+ * of range), FH_ERR_SHAPE (batch outside [1, max_batch]), FH_ERR_TIMEOUT (a kernel-side
+ * error latched by an earlier call), FH_ERR_CUDA; asynchronous on `stream`. */
 int fh_dit_block_forward(fh_dit* m, int block, const float* x_in, float* x_out,
                          const void* audio, const float* t, int batch, void* ws,
                          void* stream);
 
-/* One flow prediction at noise level sigma (timestep t = sigma):
+/* One flow prediction at noise level sigma (timestep t = sigma) (gizai:flashhead, opening
+ * paragraph: the transformer predicts the flow of the noisy latent conditioned on the
+ * reference latent; Types > FlashHead: `patch` over the concatenation [noisy | reference],
+ * the 30 blocks, the output norm modulated by `headMods` + the timestep embedding, `head`):
  * v_out = head(blocks(patch([x_noisy | ref]))), all device float32 [B, C, F, H, W];
- * audio device [B, F, A, D]. No motion pinning (the sampler does that). */
+ * audio device [B, F, A, D]. No motion pinning (the sampler does that). Errors as
+ * fh_dit_block_forward. */
 int fh_dit_predict_flow(fh_dit* m, const float* x_noisy, const float* ref,
                         const void* audio, float sigma, float* v_out, int batch,
                         void* ws, void* stream);
 
-/* The slice sampler: x starts as `noise` (frames 0-1 ignored), frames 0-1 are set
+/* The slice sampler (gizai:flashhead, opening paragraph and Methods > talk: 4 flow steps per
+ * slice, the first latent frames carrying the previous slice's motion): x starts as `noise` (frames 0-1 ignored), frames 0-1 are set
  * to `motion` before each of the `nsteps` flow predictions and on the output, and
  * each step applies x += (sigmas[s+1] - sigmas[s]) * v. sigmas: host float32
  * [nsteps + 1]. noise/ref/x_out device [B, C, F, H, W], motion device
@@ -187,7 +199,9 @@ int fh_sample_slice_host(fh_dit* m, const float* noise_host, const float* ref_ho
 int fh_audio_project(fh_dit* m, const float* states, void* tokens, int batch, void* ws, void* stream);
 
 /* Copy weight tensor `tensor_id` to host memory as float32 in its logical
- * row-major shape; `bytes` must equal 4 * element count. Synchronous. */
+ * row-major shape; `bytes` must equal 4 * element count (else FH_ERR_ARG; an unknown id
+ * is FH_ERR_ARG too). Synchronous. The pages have no such call: it exists so that a test
+ * can give the oracle the very weights the GPU uses (Types > FlashHead names the tensors). */
 int fh_dit_get_weight(const fh_dit* m, int tensor_id, void* host_dst, size_t bytes);
 
 /* Wait for `stream`, then report a latched kernel-side error (FH_ERR_TIMEOUT) and
